@@ -1,0 +1,466 @@
+"""Benchmark of the fused KV-cache step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload single_bf16|verify_bf16|long_bf16|batch_bf16]
+
+Prints ONE JSON line on rank 0.  A step is one pass of the whole hot path over
+one batch of synthetic input: for a fused-step workload the projection/RoPE/
+cache-scatter kernel then the full-cache attention; for the verify workload
+the verify pass plus the acceptance reduction.  Inputs are resident in HBM
+when the timed region starts; L2 is flushed (a 512 MB write) before every
+timed step, and each step is timed with CUDA events on the launching stream.
+Under torchrun every rank runs its own sequences (weak scaling, no data-path
+collective); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference this method
+has) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+L2_FLUSH_BYTES = 512 << 20
+DEFAULT_WORKLOAD = "single_bf16"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ helpers
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_desc(name, cfg):
+    if cfg["kind"] == "fused":
+        return (f"{name}: fused step B={cfg['B']} N={cfg['N']} D={cfg['D']} H={cfg['H']} "
+                f"dh={cfg['dh']} |Q|={cfg['n_track'] + cfg['beta_m']} ({cfg['n_track']} tracked + "
+                f"{cfg['beta_m']} front masks) {cfg['dtype']}")
+    R = cfg["n_tv"] + 2 * cfg["n_s"]
+    return (f"{name}: verify pass + acceptance B={cfg['B']} N={cfg['N']} D={cfg['D']} "
+            f"H={cfg['H']} dh={cfg['dh']} R={R} ({cfg['n_tv']} T_v + {cfg['n_s']} draft + "
+            f"{cfg['n_s']} mask rows) V={cfg['vocab']} {cfg['dtype']}")
+
+
+def algorithmic_bytes(cfg):
+    """Bytes each kernel must move at least (per launch), by its definition.
+
+    projection: W_qkv + the gathered rows x[Q] + new k, v written to the cache
+                + rotated q written for the attention;
+    attention:  the whole K, V cache of every sequence (plus side slots)
+                + q read + output written;
+    accept:     the logits."""
+    e = 2 if cfg["dtype"] == "bf16" else 4
+    B, N, D, H, dh = cfg["B"], cfg["N"], cfg["D"], cfg["H"], cfg["dh"]
+    E = H * dh
+    rows = cfg["n_track"] + cfg["beta_m"] if cfg["kind"] == "fused" else cfg["n_tv"] + 2 * cfg["n_s"]
+    M = B * rows
+    side = B * H * cfg.get("n_s", 0) * dh * e * 2 if cfg["kind"] == "verify" else 0
+    proj = 3 * E * D * e + M * D * e + 2 * M * E * e + M * E * e
+    attn = 2 * B * H * N * dh * e + side + M * E * e + M * E * e
+    out = {"proj": proj, "attn": attn}
+    if cfg["kind"] == "verify":
+        out["accept"] = M * cfg["vocab"] * 4
+    return out, rows
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    NAMES = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index):
+        self.samples = []
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                if not uuid.startswith("GPU-"):
+                    uuid = "GPU-" + uuid
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.h, self.nv = h, pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            self.ok = True
+        except Exception as e:  # no NVML: report it
+            self.err = repr(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.reasons_fn(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples[-3:]
+        mhz = [s[1] for s in inside]
+        bits = 0
+        for s in inside:
+            bits |= int(s[2])
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(n for b, n in self.NAMES.items() if bits & b),
+                "samples": len(inside)}
+
+
+def traffic_for(kernel_key):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary, or None when
+    the summary is missing or the kernel source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel_key)
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return d["bytes_per_launch"] if h == d["source_sha256_16"] else None
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, world, rank, local):
+    import kv_cache_attention_fdllm_b200 as F
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = W.CONFIGS[args.workload]
+    B = cfg["B"]
+    seqs = list(range(rank * B, (rank + 1) * B))  # each rank owns its own sequences
+    rope_base = cfg["rope_base"]
+    verify = cfg["kind"] == "verify"
+    if verify:
+        host = W.verify_inputs(cfg, seqs=seqs)
+        acc = W.accept_inputs(cfg, seqs=seqs)
+    else:
+        host = W.fused_inputs(cfg, seqs=seqs)
+    d = W.to_device(host, dev)
+    dt = d["w_qkv"].dtype
+    H, dh, N, D = cfg["H"], cfg["dh"], cfg["N"], cfg["D"]
+    if verify:
+        R = cfg["n_tv"] + 2 * cfg["n_s"]
+        S_max = cfg["n_s"]
+        ws = F.alloc_workspace(F.fdllm_verify_step_workspace_bytes(B, N, D, H, dh, R, S_max, dt), dev)
+        q = torch.empty((B, R, H, dh), dtype=dt, device=dev)
+        out = torch.empty((B, R, H * dh), dtype=dt, device=dev)
+        ad = W.to_device(acc, dev)
+        V = cfg["vocab"]
+        ws_a = F.alloc_workspace(F.fdllm_accept_workspace_bytes(B, R, V), dev)
+        top1 = torch.empty((B, R), dtype=torch.int32, device=dev)
+        conf = torch.empty((B, R), dtype=torch.float32, device=dev)
+        flags = torch.empty((B, R), dtype=torch.uint8, device=dev)
+        n_acc = torch.empty((B,), dtype=torch.int32, device=dev)
+        rows = R
+    else:
+        nq = cfg["n_track"] + cfg["beta_m"]
+        ws = F.alloc_workspace(F.fdllm_fused_step_workspace_bytes(B, N, D, H, dh, nq, dt), dev)
+        q = torch.empty((B, nq, H, dh), dtype=dt, device=dev)
+        out = torch.empty((B, nq, H * dh), dtype=dt, device=dev)
+        rows = nq
+
+    def stage_proj():
+        if verify:
+            F.fdllm_verify_qkv_rope_scatter(d["x_rows"], d["pos"], d["view"], d["w_qkv"],
+                                            d["k_cache"], d["v_cache"], d["k_side"], d["v_side"],
+                                            q, ws, rope_base=rope_base)
+        else:
+            F.fdllm_qkv_rope_scatter(d["x"], d["q_idx"], d["w_qkv"], d["k_cache"], d["v_cache"], q,
+                                     ws, rope_base=rope_base)
+
+    def stage_attn():
+        if verify:
+            F.fdllm_verify_attend(q, d["pos"], d["view"], d["rank"], d["k_cache"], d["v_cache"],
+                                  d["k_side"], d["v_side"], out, ws)
+        else:
+            F.fdllm_attend(q, d["k_cache"], d["v_cache"], out, ws)
+
+    def stage_accept():
+        F.fdllm_accept(ad["logits"], ad["kind"], ad["ref_tok"], ad["rank"], top1, conf, flags,
+                       n_acc, ws_a, eps=0.9, gamma=0.8)
+
+    stages = [("proj", stage_proj), ("attn", stage_attn)] + ([("accept", stage_accept)] if verify else [])
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def one_step(evs):
+        evs[0].record()
+        for i, (_, fn) in enumerate(stages):
+            fn()
+            evs[i + 1].record()
+
+    # warm-up (untimed)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        one_step([torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)])
+    torch.cuda.synchronize()
+    if F.fdllm_get_status(ws) != F.OK:
+        raise RuntimeError("device status set during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+           for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    launches0 = F.lib().fdllm_launch_count()
+    t0 = time.perf_counter()
+    # a long write first lets the host queue the timed steps ahead of the GPU
+    torch.empty(4 * L2_FLUSH_BYTES, dtype=torch.uint8, device=dev).fill_(0)
+    for k in range(args.steps):
+        flush.fill_(k & 0xff)
+        one_step(evs[k])
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    launches = F.lib().fdllm_launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    sampler.stop()
+
+    step_ms = [evs[k][0].elapsed_time(evs[k][-1]) for k in range(args.steps)]
+    stage_ms = {name: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)]
+                for i, (name, _) in enumerate(stages)}
+    mean_step = sum(step_ms) / len(step_ms)
+    if world > 1:
+        t = torch.tensor([mean_step], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        mean_step = float(t.item())
+    tokens_per_step = B * rows * world
+
+    # ---------------- end to end through the public call with host buffers
+    e2e = None
+    if not verify:
+        pin = {k: v.pin_memory() for k, v in host.items() if k in ("x", "q_idx")}
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        ws_e = F.alloc_workspace(ws.numel(), dev)
+        xd, qd = torch.empty_like(d["x"]), torch.empty_like(d["q_idx"])
+        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(max(3, args.steps // 4))]
+        for i in range(args.warmup + len(e2e_ev)):
+            flush.fill_(2)
+            ev = e2e_ev[i - args.warmup] if i >= args.warmup else None
+            if ev:
+                ev[0].record()
+            xd.copy_(pin["x"], non_blocking=True)
+            qd.copy_(pin["q_idx"], non_blocking=True)
+            F.fdllm_fused_step(xd, qd, d["w_qkv"], d["k_cache"], d["v_cache"], out, ws_e,
+                               rope_base=rope_base)
+            out_h.copy_(out, non_blocking=True)
+            if ev:
+                ev[1].record()
+        torch.cuda.synchronize()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / len(e2e_ev)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": tokens_per_step / (e2e_ms / 1e3), "unit": "query-tokens/s",
+               "h2d_bytes_per_step": int(pin["x"].numel() * pin["x"].element_size()
+                                         + pin["q_idx"].numel() * 4),
+               "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()),
+               "ms_per_step": e2e_ms,
+               "path": "pinned host x, q_idx -> fdllm_fused_step -> pinned host out"}
+
+    # ---------------- roofline of the dominant kernel
+    peak, peak_kind = measured_peaks()
+    alg, _ = algorithmic_bytes(cfg)
+    stage_mean = {k: sum(v) / len(v) for k, v in stage_ms.items()}
+    dom = max(stage_mean, key=stage_mean.get)
+    achieved = alg[dom] / (stage_mean[dom] / 1e3) / 1e9
+    step_bytes = sum(alg.values())
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
+                "algorithmic_bytes_per_launch": alg[dom],
+                "traffic": traffic_for(f"{args.workload}:{dom}"),
+                "ms_per_launch": stage_mean[dom]}
+
+    res = {
+        "metric": "fused-step query-tokens/s" if not verify else "verify-pass query-rows/s",
+        "value": tokens_per_step / (mean_step / 1e3),
+        "unit": "query-tokens/s" if not verify else "query-rows/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": mean_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg["dtype"], "data": "synthetic",
+        "config": {"workload": workload_desc(args.workload, cfg),
+                   "l2": "flushed before every timed step (512 MB write)",
+                   "parallelism": f"replicas x{world} (sequences sharded, no collective)"},
+        "hbm_gbs_step": step_bytes / (mean_step / 1e3) / 1e9,
+        "step_roofline_frac": step_bytes / (mean_step / 1e3) / 1e9 / peak,
+        "stage_ms": stage_mean,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": sampler.summary(t0, t1),
+    }
+    return res
+
+
+# ------------------------------------------------------------------ oracle leg
+
+def oracle_step_fn(cfg, seqs):
+    """One oracle pass over the given sequences of the workload (inputs prepared)."""
+    import oracle as O
+    H, dh, base = cfg["H"], cfg["dh"], cfg["rope_base"]
+    f = O.to_f64
+    if cfg["kind"] == "fused":
+        inp = W.fused_inputs(cfg, seqs=seqs)
+        a = (f(inp["x"]), inp["q_idx"].numpy(), f(inp["w_qkv"]), base, f(inp["k_cache"]),
+             f(inp["v_cache"]), H, dh, cfg["dtype"])
+        return lambda: O.fused_step(*a), len(seqs) * inp["q_idx"].shape[1]
+    inp = W.verify_inputs(cfg, seqs=seqs)
+    acc = W.accept_inputs(cfg, seqs=seqs)
+    a = (f(inp["x_rows"]), inp["pos"].numpy(), inp["view"].numpy(), inp["rank"].numpy(),
+         f(inp["w_qkv"]), base, f(inp["k_cache"]), f(inp["v_cache"]), f(inp["k_side"]),
+         f(inp["v_side"]), H, dh, cfg["dtype"])
+    la = (acc["logits"].numpy().astype(np.float64), acc["kind"].numpy(), acc["ref_tok"].numpy(),
+          acc["rank"].numpy(), 0.9, 0.8)
+
+    def step():
+        O.verify_step(*a)
+        O.accept(*la)
+    return step, len(seqs) * inp["pos"].shape[1]
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def time_oracle(cfg, budget_s, max_reps):
+    """Times the oracle as it stands on one sequence of the workload (a bounded sample)."""
+    step, units = oracle_step_fn(cfg, [0])
+    reps, t = 0, 0.0
+    while reps < max_reps and (reps == 0 or t < budget_s):
+        t0 = time.perf_counter()
+        step()
+        t += time.perf_counter() - t0
+        reps += 1
+    return units * reps / t, reps, units
+
+
+def run_reference(args, world, rank):
+    cfg = W.CONFIGS[args.workload]
+    budget = float(os.environ.get("FDLLM_ORACLE_BUDGET_S", "20"))
+    per_step = []
+    units = 0
+    for _ in range(max(1, args.steps)):
+        v, reps, units = time_oracle(cfg, budget / max(1, args.steps), 1)
+        per_step.append(units / v)
+        if sum(per_step) > budget * 3:
+            break
+    mean = sum(per_step) / len(per_step)
+    value = units / mean
+    unit = "query-tokens/s" if cfg["kind"] == "fused" else "query-rows/s"
+    sample = (f"one sequence (b=0) of {args.workload} per step: {units} query rows, the whole "
+              f"fp64 oracle step (projection, RoPE, cache write, full-cache attention"
+              + (", verify masks, acceptance over V logits" if cfg["kind"] == "verify" else "") + ")")
+    return {"impl": "reference", "metric": "fused-step query-tokens/s" if cfg["kind"] == "fused"
+            else "verify-pass query-rows/s", "value": value, "unit": unit, "n_gpus": world,
+            "steps": len(per_step), "warmup": 0, "ms_per_step": mean * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": workload_desc(args.workload, cfg), "l2": "n/a (host)",
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cpu_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=[k for k in W.CONFIGS if k != "tiny_fp32"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_env()
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return
+
+    if world > 1:
+        torch.distributed.init_process_group(
+            "nccl", device_id=torch.device("cuda", local),
+            timeout=__import__("datetime").timedelta(seconds=120))
+    try:
+        res = run_ours(args, world, rank, local)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            cfg = W.CONFIGS[args.workload]
+            v, reps, units = time_oracle(cfg, float(os.environ.get("FDLLM_ORACLE_BUDGET_S", "15")), 50)
+            res["cpu_baseline"] = {
+                "value": v, "unit": res["unit"], "cores": cpu_threads(), "kind": "oracle",
+                "sample": f"{reps} oracle step(s) of one sequence (b=0) of {args.workload}, "
+                          f"{units} query rows each, fp64 numpy"}
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,27 @@
+// Chooses the kernel family for each stage and sizes its scratch.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace fdllm {
+
+size_t proj_workspace_bytes(int M, int D, int H, int dh, int dtype, int num_sms) {
+  (void)D; (void)dtype; (void)num_sms;
+  return proj_simt_workspace_bytes(M, H, dh);
+}
+
+cudaError_t launch_proj(const ProjArgs& a, cudaStream_t stream) {
+  return launch_proj_simt(a, stream);
+}
+
+size_t attn_workspace_bytes(int B, int N, int H, int dh, int rows_per_seq, int S_max, int verify,
+                            int dtype, int num_sms) {
+  (void)B; (void)N; (void)H; (void)dh; (void)rows_per_seq; (void)S_max; (void)verify;
+  (void)dtype; (void)num_sms;
+  return 0;
+}
+
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream) {
+  return launch_attn_simt(a, stream);
+}
+
+}  // namespace fdllm

@@ -1,0 +1,93 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fdllm {
+
+// ----------------------------------------------------------------- acceptance
+struct AcceptPartial {
+  float m;
+  float l;
+  int idx;
+  int pad;
+};
+
+struct AcceptArgs {
+  int B, R, V, splits;
+  const float* logits;
+  const int8_t* kind;
+  const int32_t* ref_tok;
+  const int32_t* rank;
+  float eps, gamma;
+  int32_t* top1;
+  float* conf;
+  uint8_t* flags;
+  int32_t* n_accept;
+  AcceptPartial* parts;  // [B*R*splits]
+  unsigned* row_cnt;     // [B*R], zero between calls
+  unsigned* seq_cnt;     // [B], zero between calls
+};
+
+int accept_splits(int rows, int V, int num_sms);
+cudaError_t launch_accept(const AcceptArgs& a, cudaStream_t stream);
+
+// ----------------------------------------------------------------- projection
+// Rows of the projection: token m of sequence b = m / rows_per_seq.
+//   fused  (verify == 0): x row (b, q_idx[m]); RoPE position and cache slot q_idx[m].
+//   verify (verify == 1): x_rows row m; position pos[m]; view[m] chooses the
+//                         destination (0/1: cache slot pos[m]; 2: side slot).
+struct ProjArgs {
+  int B, N, D, H, dh, rows_per_seq, S_max, verify, dtype;
+  const void* x;           // fused: [B, N, D]; verify: [B, R, D]
+  const int32_t* idx;      // fused: q_idx [B, nq]; verify: pos [B, R]
+  const int8_t* view;      // verify only
+  const void* w;           // [3E, D]
+  double log2_base;
+  void* k_cache;
+  void* v_cache;
+  void* k_side;
+  void* v_side;
+  void* q_out;             // [B, rows, H, dh]
+  int* status;
+  void* ws;                // kernel scratch
+  size_t ws_bytes;
+};
+
+size_t proj_workspace_bytes(int M, int D, int H, int dh, int dtype, int num_sms);
+cudaError_t launch_proj(const ProjArgs& a, cudaStream_t stream);
+
+// ----------------------------------------------------------------- attention
+struct AttnArgs {
+  int B, N, H, dh, rows_per_seq, S_max, verify, causal_cross, dtype;
+  const void* q;           // [B, rows, H, dh]
+  const void* k_cache;
+  const void* v_cache;
+  const void* k_side;
+  const void* v_side;
+  const int32_t* pos;      // verify only
+  const int8_t* view;      // verify only
+  const int32_t* rank;     // verify only
+  void* out;               // [B, rows, H*dh]
+  int* status;
+  void* ws;
+  size_t ws_bytes;
+};
+
+size_t attn_workspace_bytes(int B, int N, int H, int dh, int rows_per_seq, int S_max, int verify,
+                            int dtype, int num_sms);
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream);
+
+// ----------------------------------------------------------------- kernel families
+size_t proj_simt_workspace_bytes(int M, int H, int dh);
+cudaError_t launch_proj_simt(const ProjArgs& a, cudaStream_t stream);
+cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t stream);
+
+// ----------------------------------------------------------------- helpers
+int device_sm_count();
+void count_launches(int n);
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace fdllm

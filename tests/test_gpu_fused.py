@@ -1,0 +1,141 @@
+"""GPU parity of the fused KV-cache step against the fp64 oracle (through the C ABI)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+from parity import (assert_close, check_cache_update, dtype_name, oracle_fused, run_fused_gpu)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def F():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import kv_cache_attention_fdllm_b200 as F
+    return F
+
+
+def _check_fused(F, inp, rope_base=10000.0, seqs_for_oracle=None, inp_oracle=None):
+    dev = W.to_device(inp)
+    k_in, v_in = inp["k_cache"].clone(), inp["v_cache"].clone()
+    out, ws, st = run_fused_gpu(F, dev, rope_base)
+    assert st == F.OK, f"device status {st}"
+    dt = dtype_name(inp["x"])
+    H, dh = inp["k_cache"].shape[1], inp["k_cache"].shape[3]
+    sel = list(range(inp["x"].shape[0])) if seqs_for_oracle is None else list(seqs_for_oracle)
+    ref_inp = inp if inp_oracle is None else inp_oracle
+    if inp_oracle is None and seqs_for_oracle is not None:
+        ref_inp = {k: v[sel] for k, v in inp.items() if k != "w_qkv"}
+        ref_inp["w_qkv"] = inp["w_qkv"]
+    K2, V2, ref_out = oracle_fused(ref_inp, H, dh, rope_base, dt)
+    out_c = out.cpu()[sel]
+    err = assert_close(O.to_f64(out_c), ref_out, dt, "attention output")
+    qi = ref_inp["q_idx"].numpy()
+    check_cache_update(dev["k_cache"].cpu()[sel], k_in[sel], K2, qi, dt, "k_cache")
+    check_cache_update(dev["v_cache"].cpu()[sel], v_in[sel], V2, qi, dt, "v_cache")
+    return err, out, dev
+
+
+def test_tiny_fp32_config(F):
+    cfg = W.CONFIGS["tiny_fp32"]
+    _check_fused(F, W.fused_inputs(cfg), cfg["rope_base"])
+
+
+def test_single_bf16_config(F):
+    cfg = W.CONFIGS["single_bf16"]
+    _check_fused(F, W.fused_inputs(cfg), cfg["rope_base"])
+
+
+def test_long_bf16_config(F):
+    cfg = W.CONFIGS["long_bf16"]
+    _check_fused(F, W.fused_inputs(cfg), cfg["rope_base"])
+
+
+def test_batch_bf16_config_sampled(F):
+    """Full-size B=64 batch; the oracle recomputes sampled sequences one by one
+    from their own input substreams (the first, a middle one, the last)."""
+    cfg = W.CONFIGS["batch_bf16"]
+    inp = W.fused_inputs(cfg)
+    seqs = [0, 37, 63]
+    _check_fused(F, inp, cfg["rope_base"], seqs_for_oracle=seqs,
+                 inp_oracle=W.fused_inputs(cfg, seqs=seqs))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("dh", [64, 128])
+@pytest.mark.parametrize("shape", [(2, 200, 128, 2, 5), (1, 130, 256, 3, 1), (3, 385, 192, 1, 37)])
+def test_ragged_shapes(F, dtype, dh, shape):
+    """Several KV tiles with a ragged tail, ragged query counts, B > 1."""
+    B, N, D, H, nq = shape
+    inp = W.random_fused(B, N, D, H, dh, nq=nq, dtype=dtype, seed=hash((shape, dh)) % 1000)
+    _check_fused(F, inp)
+
+
+def test_edge_slots_and_single_query(F):
+    N = 257
+    q_idx = np.array([[0, N - 1, 128], [N - 1, 5, 0]], np.int32)
+    _check_fused(F, W.random_fused(2, N, 128, 2, 128, q_idx=q_idx, seed=5))
+    _check_fused(F, W.random_fused(1, N, 128, 2, 128, q_idx=np.array([[N - 1]]), seed=6))
+
+
+def test_query_set_covers_whole_cache(F):
+    N = 96
+    q_idx = np.stack([np.random.default_rng(1).permutation(N)]).astype(np.int32)
+    _check_fused(F, W.random_fused(1, N, 64 * 2, 2, 64, q_idx=q_idx, seed=7))
+
+
+def test_rows_outside_q_are_never_read(F):
+    """x rows outside Q are NaN: the step must not use them."""
+    inp = W.random_fused(2, 300, 128, 2, 128, nq=9, seed=8, x_outside=float("nan"))
+    _, out, _ = _check_fused(F, inp)
+    assert torch.isfinite(out).all()
+
+
+def test_deterministic(F):
+    inp = W.random_fused(2, 700, 256, 4, 128, nq=33, seed=9)
+    a = W.to_device(inp)
+    b = W.to_device(inp)
+    oa, _, _ = run_fused_gpu(F, a, 10000.0)
+    ob, _, _ = run_fused_gpu(F, b, 10000.0)
+    assert torch.equal(oa, ob) and torch.equal(a["k_cache"], b["k_cache"])
+
+
+def test_out_of_range_index_sets_status_and_skips_row(F):
+    inp = W.random_fused(1, 100, 128, 2, 64, q_idx=np.array([[3, 100, 7]]), seed=10)
+    dev = W.to_device(inp)
+    k_in = dev["k_cache"].clone()
+    out, ws, st = run_fused_gpu(F, dev, 10000.0)
+    assert st == F.ERR_BAD_INDEX
+    changed = (dev["k_cache"] != k_in).any(dim=3).any(dim=1)[0]
+    assert set(torch.nonzero(changed).flatten().tolist()) <= {3, 7}
+    assert F.fdllm_get_status(ws) == F.OK  # read-and-clear
+
+
+def test_empty_batch_is_a_no_op(F):
+    x = torch.zeros((0, 10, 64), dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros((0, 2), dtype=torch.int32, device="cuda")
+    w = torch.zeros((3 * 64, 64), dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros((0, 1, 10, 64), dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros((0, 2, 64), dtype=torch.bfloat16, device="cuda")
+    ws = F.alloc_workspace(4096, "cuda")
+    F.fdllm_fused_step(x, q, w, k, k.clone(), out, ws)
+    assert F.fdllm_get_status(ws) == F.OK
+
+
+def test_stage_calls_equal_fused_call(F):
+    inp = W.random_fused(2, 300, 256, 2, 128, nq=11, seed=12)
+    a, b = W.to_device(inp), W.to_device(inp)
+    out_f, _, _ = run_fused_gpu(F, a, 500.0)
+    B, N, D = b["x"].shape
+    H, dh, nq = 2, 128, 11
+    ws = F.alloc_workspace(F.fdllm_fused_step_workspace_bytes(B, N, D, H, dh, nq, torch.bfloat16), "cuda")
+    q = torch.empty((B, nq, H, dh), dtype=torch.bfloat16, device="cuda")
+    out_s = torch.empty_like(out_f)
+    F.fdllm_qkv_rope_scatter(b["x"], b["q_idx"], b["w_qkv"], b["k_cache"], b["v_cache"], q, ws,
+                             rope_base=500.0)
+    F.fdllm_attend(q, b["k_cache"], b["v_cache"], out_s, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out_f, out_s) and torch.equal(a["k_cache"], b["k_cache"])

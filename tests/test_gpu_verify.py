@@ -1,0 +1,96 @@
+"""GPU parity of the Flash-Verify pass against the fp64 oracle (through the C ABI)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+from parity import assert_close, dtype_name, oracle_verify, run_verify_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def F():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import kv_cache_attention_fdllm_b200 as F
+    return F
+
+
+def _check_verify(F, inp, rope_base=10000.0, causal=False, seqs=None, inp_oracle=None):
+    dev = W.to_device(inp)
+    k_in, v_in = inp["k_cache"].clone(), inp["v_cache"].clone()
+    out, ws, st = run_verify_gpu(F, dev, rope_base, causal)
+    assert st == F.OK, f"device status {st}"
+    dt = dtype_name(inp["x_rows"])
+    H, dh = inp["k_cache"].shape[1], inp["k_cache"].shape[3]
+    sel = list(range(inp["x_rows"].shape[0])) if seqs is None else list(seqs)
+    ref_inp = inp if inp_oracle is None else inp_oracle
+    K2, V2, KS, VS, ref_out = oracle_verify(ref_inp, H, dh, rope_base, dt, causal)
+    assert_close(O.to_f64(out.cpu()[sel]), ref_out, dt, "verify output")
+    kc, vc = dev["k_cache"].cpu()[sel], dev["v_cache"].cpu()[sel]
+    pos, view = ref_inp["pos"].numpy(), ref_inp["view"].numpy()
+    N = kc.shape[2]
+    for i in range(len(sel)):
+        written = np.zeros(N, bool)
+        written[pos[i][(view[i] == 0) | (view[i] == 1)]] = True
+        keep = torch.from_numpy(~written)
+        assert torch.equal(kc[i][:, keep], k_in[sel[i]][:, keep])
+        assert torch.equal(vc[i][:, keep], v_in[sel[i]][:, keep])
+        assert_close(O.to_f64(kc[i][:, torch.from_numpy(written)]), K2[i][:, written], dt, "k written")
+        assert_close(O.to_f64(vc[i][:, torch.from_numpy(written)]), V2[i][:, written], dt, "v written")
+        n_side = int((view[i] == 2).sum())
+        ks, vs = dev["k_side"].cpu()[sel[i]], dev["v_side"].cpu()[sel[i]]
+        assert_close(O.to_f64(ks[:, :n_side]), KS[i][:, :n_side], dt, "k side")
+        assert_close(O.to_f64(vs[:, :n_side]), VS[i][:, :n_side], dt, "v side")
+        assert torch.equal(ks[:, n_side:], inp["k_side"][sel[i]][:, n_side:])
+    return out
+
+
+def test_verify_bf16_config_sampled(F):
+    cfg = W.CONFIGS["verify_bf16"]
+    inp = W.verify_inputs(cfg)
+    seqs = [0, 5]
+    _check_verify(F, inp, cfg["rope_base"], seqs=seqs, inp_oracle=W.verify_inputs(cfg, seqs=seqs))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dtype,dh", [("bf16", 128), ("bf16", 64), ("f32", 64)])
+def test_verify_ragged(F, causal, dtype, dh):
+    inp = W.random_verify(2, 333, 128, 2, dh, n_tv=5, n_s=7, S_max=9, dtype=dtype, seed=21)
+    _check_verify(F, inp, causal=causal)
+
+
+def test_verify_many_views_spanning_tiles(F):
+    inp = W.random_verify(1, 1000, 128, 2, 128, n_tv=3, n_s=70, S_max=140, seed=22)
+    _check_verify(F, inp)
+    _check_verify(F, inp, causal=True)
+
+
+def test_verify_without_views_equals_fused(F):
+    inp = W.random_verify(2, 250, 128, 2, 128, n_tv=6, n_s=0, S_max=0, seed=23, with_views=False)
+    out_v = _check_verify(F, inp)
+    fin = dict(x=torch.zeros((2, 250, 128), dtype=torch.bfloat16), q_idx=inp["pos"],
+               w_qkv=inp["w_qkv"], k_cache=inp["k_cache"], v_cache=inp["v_cache"])
+    for b in range(2):
+        fin["x"][b, inp["pos"][b].long()] = inp["x_rows"][b]
+    from parity import run_fused_gpu
+    dev = W.to_device(fin)
+    out_f, _, st = run_fused_gpu(F, dev, 10000.0)
+    assert st == F.OK
+    assert torch.equal(out_f, out_v)
+
+
+def test_single_s_position_modes_coincide(F):
+    inp = W.random_verify(2, 200, 128, 2, 128, n_tv=2, n_s=1, seed=24)
+    a = _check_verify(F, inp, causal=False)
+    b = _check_verify(F, inp, causal=True)
+    assert torch.equal(a, b)
+
+
+def test_side_overflow_sets_status(F):
+    inp = W.random_verify(1, 120, 128, 2, 64, n_tv=2, n_s=5, S_max=3, seed=25)
+    dev = W.to_device(inp)
+    out, ws, st = run_verify_gpu(F, dev, 10000.0)
+    assert st == F.ERR_BAD_INDEX

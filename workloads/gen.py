@@ -239,3 +239,70 @@ def to_device(inputs: dict, device="cuda") -> dict:
     """Copy every tensor of an input dict to `device` (other values unchanged)."""
     return {k: (v.to(device).contiguous() if isinstance(v, torch.Tensor) else v)
             for k, v in inputs.items()}
+
+
+# ---------------------------------------------------------------------------
+# general shapes for edge-case tests (same distributions, any sizes)
+
+def random_fused(B, N, D, H, dh, nq=None, q_idx=None, dtype="bf16", seed=100, x_outside=0.0):
+    """A fused-step input of any shape.  q_idx (int array [B, nq]) may be given;
+    otherwise nq distinct slots per sequence are drawn uniformly from [0, N).
+    Rows of x outside Q are filled with x_outside (NaN poisons them)."""
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 77])))
+    if q_idx is None:
+        q_idx = np.stack([g.choice(N, nq, replace=False) for _ in range(B)]).astype(np.int32)
+    q_idx = np.asarray(q_idx, np.int32)
+    nq = q_idx.shape[1]
+    x = np.full((B, N, D), x_outside, np.float32)
+    for b in range(B):
+        ok = (q_idx[b] >= 0) & (q_idx[b] < N)
+        x[b, q_idx[b][ok]] = g.standard_normal((int(ok.sum()), D), dtype=np.float32)
+    E = H * dh
+    w = g.standard_normal((3 * E, D), dtype=np.float32) / np.float32(math.sqrt(D))
+    k = g.standard_normal((B, H, N, dh), dtype=np.float32)
+    v = g.standard_normal((B, H, N, dh), dtype=np.float32)
+    return dict(x=_store(x, dtype), q_idx=torch.from_numpy(q_idx), w_qkv=_store(w, dtype),
+                k_cache=_store(k, dtype), v_cache=_store(v, dtype))
+
+
+def random_verify(B, N, D, H, dh, n_tv, n_s, S_max=None, dtype="bf16", seed=200,
+                  with_views=True):
+    """A verify-pass input of any shape: rows [T_v (n_tv) | draft (n_s) | mask (n_s)]
+    at distinct random positions, ranks a random permutation per sequence."""
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 78])))
+    S_max = n_s if S_max is None else S_max
+    R = n_tv + (2 * n_s if with_views else 0)
+    pos = np.empty((B, R), np.int32)
+    view = np.empty((B, R), np.int8)
+    rank = np.empty((B, R), np.int32)
+    for b in range(B):
+        p = g.choice(N, n_tv + n_s, replace=False)
+        T, S = p[:n_tv], p[n_tv:]
+        r = g.permutation(n_s)
+        if with_views:
+            pos[b] = np.concatenate([T, S, S])
+            view[b] = [0] * n_tv + [1] * n_s + [2] * n_s
+            rank[b] = np.concatenate([np.full(n_tv, -1), r, r])
+        else:
+            pos[b], view[b], rank[b] = T, 0, -1
+    x_rows = g.standard_normal((B, R, D), dtype=np.float32)
+    E = H * dh
+    w = g.standard_normal((3 * E, D), dtype=np.float32) / np.float32(math.sqrt(D))
+    k = g.standard_normal((B, H, N, dh), dtype=np.float32)
+    v = g.standard_normal((B, H, N, dh), dtype=np.float32)
+    ks = g.standard_normal((B, H, max(S_max, 1), dh), dtype=np.float32)[:, :, :S_max]
+    vs = g.standard_normal((B, H, max(S_max, 1), dh), dtype=np.float32)[:, :, :S_max]
+    return dict(x_rows=_store(x_rows, dtype), pos=torch.from_numpy(pos),
+                view=torch.from_numpy(view), rank=torch.from_numpy(rank), w_qkv=_store(w, dtype),
+                k_cache=_store(k, dtype), v_cache=_store(v, dtype), k_side=_store(ks, dtype),
+                v_side=_store(vs, dtype), S_max=S_max)
+
+
+def random_logits(B, R, V, seed=300, spike_lo=2.0, spike_hi=12.0):
+    """fp32 logits [B, R, V]: N(0,1) plus one spike of U(spike_lo, spike_hi) per row."""
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 79])))
+    l = g.standard_normal((B, R, V), dtype=np.float32)
+    tok = g.integers(0, V, (B, R))
+    l[np.arange(B)[:, None], np.arange(R)[None, :], tok] += g.uniform(
+        spike_lo, spike_hi, (B, R)).astype(np.float32)
+    return torch.from_numpy(l), tok.astype(np.int32)
