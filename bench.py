@@ -176,7 +176,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     cfg = W.CONFIGS[args.workload]
     B = cfg["B"]
-    seqs = list(range(rank * B, (rank + 1) * B))  # each rank owns its own sequences
+    seqs = F.rank_sequences(B, rank)  # each rank owns its own sequences
     rope_base = cfg["rope_base"]
     verify = cfg["kind"] == "verify"
     if verify:
@@ -269,11 +269,7 @@ def run_ours(args, world, rank, local):
     step_ms = [evs[k][0].elapsed_time(evs[k][-1]) for k in range(args.steps)]
     stage_ms = {name: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)]
                 for i, (name, _) in enumerate(stages)}
-    mean_step = sum(step_ms) / len(step_ms)
-    if world > 1:
-        t = torch.tensor([mean_step], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        mean_step = float(t.item())
+    mean_step = F.max_over_ranks(sum(step_ms) / len(step_ms), dev)
     tokens_per_step = B * rows * world
 
     # ---------------- end to end through the public call with host buffers
@@ -298,11 +294,7 @@ def run_ours(args, world, rank, local):
             if ev:
                 ev[1].record()
         torch.cuda.synchronize()
-        e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / len(e2e_ev)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = F.max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / len(e2e_ev), dev)
         e2e = {"value": tokens_per_step / (e2e_ms / 1e3), "unit": "query-tokens/s",
                "h2d_bytes_per_step": int(pin["x"].numel() * pin["x"].element_size()
                                          + pin["q_idx"].numel() * 4),

@@ -16,5 +16,7 @@ from .api import (ERR_BAD_INDEX, ERR_CUDA, ERR_INVALID_ARG, ERR_TIMEOUT, ERR_UNS
                   fdllm_qkv_rope_scatter, fdllm_verify_attend, fdllm_verify_qkv_rope_scatter,
                   fdllm_verify_step, fdllm_verify_step_workspace_bytes)
 
+from .shard import max_over_ranks, rank_sequences  # noqa: E402
+
 __all__ = [n for n in dir() if n.startswith(("fdllm_", "FLAG_", "ERR_"))] + [
-    "OK", "FdllmError", "alloc_workspace", "lib", "LIB_PATH"]
+    "OK", "FdllmError", "alloc_workspace", "lib", "LIB_PATH", "max_over_ranks", "rank_sequences"]
