@@ -180,6 +180,34 @@ fdllm_status fdllm_accept(int B, int R, int V, const float* logits, const int8_t
                           int32_t* top1, float* conf, uint8_t* flags, int32_t* n_accept,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* Size of the device array that fdllm_accept_noalloc uses as its scratch. */
+#define FDLLM_ACCEPT_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* fdllm_accept without a workspace.  The paper has no counterpart: this entry
+ * point exists for callers that cannot allocate device memory where they call
+ * the library, e.g. a plugin that its host hands only the input and output
+ * buffers, a runtime that reserved all device memory for its own pool up front,
+ * or a latency-critical loop where a cudaMalloc would synchronise the device.
+ *   Arguments and results are those of fdllm_accept (same kernel, same rows),
+ *   minus the workspace.  The call allocates nothing (no cudaMalloc, no
+ *   cudaFree, no allocating library routine).  Its scratch is a device array of
+ *   FDLLM_ACCEPT_NOALLOC_SCRATCH_BYTES compiled into the library: every GPU that
+ *   loads the library holds it until the process exits.  It needs
+ *   align256(B*R*splits*16) + align256(B*R*4) + align256(B*4) bytes, where
+ *   splits <= max(1, 8*SMs / (B*R)); B*R <= 131072 always fits, and a call that
+ *   does not fit returns FDLLM_ERR_UNSUPPORTED without launching anything.
+ *   Every call on a device shares the one array, which keeps the last call's
+ *   contents; each call first clears (cudaMemsetAsync on `stream`) the counters
+ *   that must start at zero.  Calls that overlap on the GPU (on different
+ *   streams, or from several threads) race on the array: order them.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture. */
+fdllm_status fdllm_accept_noalloc(int B, int R, int V, const float* logits, const int8_t* kind,
+                                  const int32_t* ref_tok, const int32_t* rank, float eps,
+                                  float gamma, int32_t* top1, float* conf, uint8_t* flags,
+                                  int32_t* n_accept, void* stream);
+
 /* Number of kernels this library has launched in this process (a diagnostic
  * counter, incremented on the host at every launch; never reset). */
 uint64_t fdllm_launch_count(void);

@@ -11,7 +11,8 @@ lib()  # fail loudly at import when the CUDA library is missing
 
 from .api import (ERR_BAD_INDEX, ERR_CUDA, ERR_INVALID_ARG, ERR_TIMEOUT, ERR_UNSUPPORTED,  # noqa: E402
                   ERR_WORKSPACE, FLAG_ACCEPT, FLAG_COMMIT, FLAG_PASS, OK, FdllmError,
-                  alloc_workspace, fdllm_accept, fdllm_accept_workspace_bytes, fdllm_attend,
+                  alloc_workspace, fdllm_accept, fdllm_accept_noalloc,
+                  fdllm_accept_workspace_bytes, fdllm_attend,
                   fdllm_fused_step, fdllm_fused_step_workspace_bytes, fdllm_get_status,
                   fdllm_qkv_rope_scatter, fdllm_verify_attend, fdllm_verify_qkv_rope_scatter,
                   fdllm_verify_step, fdllm_verify_step_workspace_bytes)

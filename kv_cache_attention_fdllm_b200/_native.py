@@ -32,6 +32,8 @@ SIGNATURES = {
                                                     _c_int, _vp, _c_size, _vp]),
     "fdllm_accept": (_c_int, [_c_int] * 3 + [_vp, _vp, _vp, _vp, _c_float, _c_float, _vp, _vp,
                                              _vp, _vp, _vp, _c_size, _vp]),
+    "fdllm_accept_noalloc": (_c_int, [_c_int] * 3 + [_vp, _vp, _vp, _vp, _c_float, _c_float,
+                                                     _vp, _vp, _vp, _vp, _vp]),
     "fdllm_launch_count": (ctypes.c_uint64, []),
     "fdllm_get_status": (_c_int, [_vp, _vp]),
 }

@@ -239,6 +239,30 @@ def fdllm_accept(logits, kind, ref_tok, rank, top1, conf, flags, n_accept, works
     return top1, conf, flags, n_accept
 
 
+def fdllm_accept_noalloc(logits, kind, ref_tok, rank, top1, conf, flags, n_accept, eps=0.9,
+                         gamma=0.8, stream=None):
+    """fdllm_accept without a workspace, for callers that cannot allocate device
+    memory where they call the library (see include/fdllm.h): the scratch is a
+    fixed device array inside the library, shared by every call on a device."""
+    _need(logits, "logits", torch.float32)
+    B, R, V = logits.shape
+    dev = logits.device
+    _need(kind, "kind", torch.int8, (B, R), dev)
+    if ref_tok is not None:
+        _need(ref_tok, "ref_tok", torch.int32, (B, R), dev)
+    if rank is not None:
+        _need(rank, "rank", torch.int32, (B, R), dev)
+    _need(top1, "top1", torch.int32, (B, R), dev)
+    _need(conf, "conf", torch.float32, (B, R), dev)
+    _need(flags, "flags", torch.uint8, (B, R), dev)
+    _need(n_accept, "n_accept", torch.int32, (B,), dev)
+    st = lib().fdllm_accept_noalloc(B, R, V, _p(logits), _p(kind), _p(ref_tok), _p(rank),
+                                    float(eps), float(gamma), _p(top1), _p(conf), _p(flags),
+                                    _p(n_accept), _stream(stream))
+    _check(st, "fdllm_accept_noalloc")
+    return top1, conf, flags, n_accept
+
+
 def fdllm_get_status(workspace, stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device status word."""
     return int(lib().fdllm_get_status(_p(workspace), _stream(stream)))

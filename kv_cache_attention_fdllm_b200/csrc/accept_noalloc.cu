@@ -1,0 +1,93 @@
+// fdllm_accept_noalloc: the acceptance reduction without a caller workspace.
+//
+// Some host programs cannot allocate device memory at the point where they
+// call this library: a plugin that an inference server hands only its input
+// and output buffers, a runtime that reserved all device memory up front for
+// its own pool, or a latency-critical loop where a cudaMalloc would
+// synchronise the device.  For them this entry point keeps the reduction's
+// scratch (per-split partials and the last-arriver counters) in a fixed
+// device array compiled into the library, so the call allocates nothing.
+//
+// The array is file-scope and static: every GPU that loads the library holds
+// it until the process exits.  Host code only sees a host-side stand-in under
+// its name, so the device address is looked up once per device with
+// cudaGetSymbolAddress (on the first call, with that device current) and that
+// address is what the kernel receives.
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+constexpr size_t kScratchBytes = FDLLM_ACCEPT_NOALLOC_SCRATCH_BYTES;
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_accept_scratch[kScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_dev_ptr[kMaxDevices];  // device address of g_accept_scratch, per device
+
+// Device address of the scratch array on the current device (set-up on first use).
+fdllm_status scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FDLLM_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FDLLM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_dev_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_accept_scratch);
+    if (e != cudaSuccess || p == nullptr) return FDLLM_ERR_CUDA;
+    g_scratch_dev_ptr[dev] = p;
+  }
+  *out = g_scratch_dev_ptr[dev];
+  return FDLLM_OK;
+}
+
+bool is_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" fdllm_status fdllm_accept_noalloc(int B, int R, int V, const float* logits,
+                                             const int8_t* kind, const int32_t* ref_tok,
+                                             const int32_t* rank, float eps, float gamma,
+                                             int32_t* top1, float* conf, uint8_t* flags,
+                                             int32_t* n_accept, void* stream) {
+  using namespace fdllm;
+  if (B < 0 || R < 0 || V < 1) return FDLLM_ERR_INVALID_ARG;
+  if ((long long)B * R > (1ll << 31) - 1 || (long long)B * R * V > (1ll << 40))
+    return FDLLM_ERR_UNSUPPORTED;
+  const int rows = B * R;
+  const int splits = accept_splits(rows, V, device_sm_count());
+  // scratch layout: [partials | per-row counters | per-sequence counters]
+  const size_t parts_bytes = align_up((size_t)rows * splits * sizeof(AcceptPartial), 256);
+  const size_t row_cnt_bytes = align_up((size_t)rows * sizeof(unsigned), 256);
+  const size_t seq_cnt_bytes = align_up((size_t)(B > 0 ? B : 1) * sizeof(unsigned), 256);
+  if (parts_bytes + row_cnt_bytes + seq_cnt_bytes > kScratchBytes) return FDLLM_ERR_UNSUPPORTED;
+  if (rows == 0) return FDLLM_OK;
+  if (!logits || !kind || !top1 || !conf || !flags || !n_accept) return FDLLM_ERR_INVALID_ARG;
+  if (!is_aligned16(logits) || !is_aligned16(kind) || !is_aligned16(top1) ||
+      !is_aligned16(conf) || !is_aligned16(flags) || !is_aligned16(n_accept))
+    return FDLLM_ERR_INVALID_ARG;
+  if ((ref_tok && !is_aligned16(ref_tok)) || (rank && !is_aligned16(rank)))
+    return FDLLM_ERR_INVALID_ARG;
+
+  void* base = nullptr;
+  fdllm_status st = scratch_address(&base);
+  if (st != FDLLM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* p = static_cast<char*>(base);
+  // the counters must start at zero; the array keeps whatever the last call left
+  if (cudaMemsetAsync(p + parts_bytes, 0, row_cnt_bytes + seq_cnt_bytes, s) != cudaSuccess)
+    return FDLLM_ERR_CUDA;
+
+  AcceptArgs a{};
+  a.B = B; a.R = R; a.V = V; a.splits = splits;
+  a.logits = logits; a.kind = kind; a.ref_tok = ref_tok; a.rank = rank;
+  a.eps = eps; a.gamma = gamma;
+  a.top1 = top1; a.conf = conf; a.flags = flags; a.n_accept = n_accept;
+  a.parts = reinterpret_cast<AcceptPartial*>(p);
+  a.row_cnt = reinterpret_cast<unsigned*>(p + parts_bytes);
+  a.seq_cnt = reinterpret_cast<unsigned*>(p + parts_bytes + row_cnt_bytes);
+  return launch_accept(a, s) == cudaSuccess ? FDLLM_OK : FDLLM_ERR_CUDA;
+}
