@@ -15,7 +15,7 @@
  *   fdllm_verify_step  the Flash-Verify pass ([review] "Flash-Verify", sec. 2.3,
  *                      Fig. 2; "How It Works", Step 1: Verification): rows
  *                      [T_v | draft view of S | mask view of S]; the two views share
- *                      positions (RoPE) but cannot see each other.
+ *                      positions (RoPE) while each is hidden from the other.
  *   fdllm_accept       per-row top-1 and confidence, the epsilon split D_t / S_t
  *                      and the gamma prefix acceptance up to the first mismatch
  *                      ([review] "Flash-Verify", sec. 2.3 and the worked example).
@@ -132,7 +132,7 @@ fdllm_status fdllm_attend(int B, int N, int H, int dh, int nq, int dtype, const 
  *   write theirs into side slots 0, 1, ... in row order (at most S_max of them),
  *   so the cache never holds mask-view keys.  Visibility:
  *     view 0/1 rows: every cache slot, no side slot;
- *     view 2 rows, causal_cross = 0 (the pages' "cannot see each other"):
+ *     view 2 rows, causal_cross = 0 (the two views mutually hidden, the default):
  *       every cache slot except the draft-view positions, and every side slot;
  *     view 2 rows, causal_cross = 1 (reading of [review] Appx. C, Remark 1):
  *       the draft key at a position of smaller rank and the mask key at a

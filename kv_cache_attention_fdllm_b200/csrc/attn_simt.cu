@@ -3,7 +3,7 @@
 // Flash-dLLM review, "How It Works", Step 1: Draft: after the new k, v are
 // written, every query attends over the whole bidirectional cache.  With the
 // verify metadata it applies the Flash-Verify view rule ("Flash-Verify",
-// sec. 2.3): draft and mask views share positions but cannot see each other.
+// sec. 2.3): draft and mask views share positions, each hidden from the other.
 //
 // One CTA (4 warps) per (sequence, head, group of 4 query rows).  Warps take
 // keys round-robin; the lanes of a warp split the head dimension, so each key

@@ -21,7 +21,7 @@ What is computed (each function states its passage):
   * verify_step  - the Flash-Verify pass ([review], "Flash-Verify", sec. 2.3,
                    Fig. 2; "How It Works", Step 1: Verification): rows
                    [T_v | draft view | mask view]; the two views share
-                   positions but cannot see each other.
+                   positions, and neither view attends to the other's keys.
   * accept       - top-1 / confidence, the epsilon split into D_t / S_t and the
                    gamma prefix acceptance ([review], "Flash-Verify", sec. 2.3
                    and the worked example).
@@ -133,9 +133,9 @@ def project_qkv(x_rows: np.ndarray, w_qkv: np.ndarray, H: int, dh: int):
 def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, visible: np.ndarray | None = None):
     """softmax(q K^T / sqrt(dh)) V for one head: q [nq, dh], K, V [Nk, dh].
 
-    visible [nq, Nk] (optional) removes keys a row may not see.  Full
-    bidirectional attention otherwise ([review], "How It Works": the draft
-    pass attends over the full cache)."""
+    visible [nq, Nk] (optional) removes keys a row may not see.  Otherwise
+    every query sees every key ([review], "How It Works": the draft pass
+    attends over the whole cache)."""
     dh = q.shape[-1]
     s = (q @ K.T) / np.sqrt(dh)
     if visible is not None:
@@ -181,7 +181,7 @@ def verify_visibility(view, rank, n_cache_pos, draft_pos, causal_cross=False):
 
     Keys are the N cache slots followed by the side slots that hold the
     mask-view k,v (one per mask-view row, in row order).  The draft view and
-    the mask view share positions but cannot see each other ([review],
+    the mask view share positions while each is hidden from the other ([review],
     "Flash-Verify", sec. 2.3, Fig. 2; "How It Works", Step 1: Verification):
       * view 0 (T_v) and view 1 (draft) rows see every cache slot, including
         the draft-view k,v written at the S positions, and no side slot;
