@@ -5,11 +5,12 @@
 namespace fdllm {
 
 size_t proj_workspace_bytes(int M, int D, int H, int dh, int dtype, int num_sms) {
-  (void)D; (void)dtype; (void)num_sms;
+  if (dtype == FDLLM_BF16) return proj_tc_workspace_bytes(M, D, H, dh, num_sms);
   return proj_simt_workspace_bytes(M, H, dh);
 }
 
 cudaError_t launch_proj(const ProjArgs& a, cudaStream_t stream) {
+  if (a.dtype == FDLLM_BF16) return launch_proj_tc(a, stream);
   return launch_proj_simt(a, stream);
 }
 

@@ -82,6 +82,8 @@ cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream);
 
 // ----------------------------------------------------------------- kernel families
 size_t proj_simt_workspace_bytes(int M, int H, int dh);
+size_t proj_tc_workspace_bytes(int M, int D, int H, int dh, int num_sms);
+cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream);
 cudaError_t launch_proj_simt(const ProjArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t stream);
 

@@ -1,0 +1,565 @@
+// QKV projection + RoPE + cache scatter on the 5th-generation tensor cores (bf16).
+//
+// Flash-dLLM review, "How It Works", Step 1: Draft (Alg. 1): the step reads only
+// the hidden rows x[Q], builds q, k, v on chip and writes k, v into the cache at
+// exactly the slots of Q.
+//
+// Shape of the work: Y = x[Q] * W^T with few rows (B*|Q| = 32..2048) and a wide
+// W (3E x D = 12288 x 4096, 100 MB), so for small batches the kernel streams W
+// once from HBM.  It is computed transposed (swap-AB): Y^T[128 features x BN
+// tokens] = W_tile[128 x K] * X[BN x K]^T, so W rows fill the MMA's M = 128 and
+// the gathered tokens are its N (16..256).
+//
+// Two kernels, the second launched as a programmatic dependent of the first:
+//   proj_prep    one CTA per row: packs x[Q] into the workspace (fused step;
+//                verify rows arrive packed) and tabulates the RoPE cos/sin of
+//                the row's position, so the epilogue does no transcendental
+//                math.  It lets the projection start at once.
+//   proj_tc      persistent stream-K GEMM.  Its W loads do not depend on the
+//                prep kernel and are issued before the grid-dependency wait.
+//
+// Persistent stream-K: one CTA per SM.  The (tile, k-step) units are laid out
+// tile after tile and every CTA takes an equal contiguous range of them, so the
+// load is balanced whatever the tile count.  A CTA's range covers whole tiles
+// and at most one partial tile at each end; a partial tile is written as an
+// fp32 partial and the last of its contributors (atomic counter) sums the
+// partials in k order (results do not depend on timing) and runs the epilogue.
+// No CTA ever waits on another.  A k-step loads `subs` 64-wide sub-blocks at
+// once (up to 512 contiguous bytes of every W row).
+//
+//   warp 0      TMA producer: W boxes [64 x 128] and X boxes [64 x BN]
+//   warp 1      TMEM allocation; lane 0 issues tcgen05.mma into one of two
+//               TMEM accumulators (the epilogue drains the other)
+//   warps 2-5   epilogue: TMEM (or the summed partials) -> shared memory ->
+//               RoPE on the q and k heads -> 16-byte stores of q, k, v rows
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+#include "tmap.h"
+
+namespace fdllm {
+
+namespace {
+
+constexpr int kBM = 128;            // W rows (features) per tile = MMA M
+constexpr int kSub = 64;            // bf16 K elements per sub-block = one 128-byte swizzle row
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr int kChunk = 32;          // tokens per epilogue pass
+constexpr int kPitch = kChunk + 1;  // staging pitch (floats)
+constexpr int kMaxBN = 256;
+constexpr uint32_t kASubBytes = kBM * kSub * 2;  // 16 KB
+
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+struct ProjTcParams {
+  int M, F, D, E, N, H, dh, rows_per_seq, S_max, verify;
+  int BN, n_tt, tiles, nks, subs, nsub_total, nstage;
+  long long total_units;
+  const int32_t* idx;
+  const int8_t* view;
+  const float2* rope_tab;  // [M][dh/2] (cos, sin) of the row's position
+  __nv_bfloat16* k_cache;
+  __nv_bfloat16* v_cache;
+  __nv_bfloat16* k_side;
+  __nv_bfloat16* v_side;
+  __nv_bfloat16* q_out;
+  int* status;
+  float* partials;     // [grid][2][BN][128]
+  unsigned* tile_cnt;  // [tiles], zero between calls
+};
+
+__device__ __forceinline__ long long unit_lo(long long total, int G, int c) {
+  return total * c / G;
+}
+// The CTA whose unit range holds unit u.
+__device__ __forceinline__ int owner_of(long long u, long long total, int G) {
+  int c = (int)(((u + 1) * G - 1) / total);
+  if (c >= G) c = G - 1;
+  while (c > 0 && unit_lo(total, G, c) > u) --c;
+  while (c + 1 < G && unit_lo(total, G, c + 1) <= u) ++c;
+  return c;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// One CTA per projection row m: xq[m] = x[b, q_idx[m]] (fused step; zeros when
+// the index is out of range) and rope_tab[m][j] = (cos, sin)(pos * theta_j).
+__global__ void __launch_bounds__(128) proj_prep_kernel(const __nv_bfloat16* __restrict__ x,
+                                                        const int32_t* __restrict__ idx, int N,
+                                                        int D, int rows_per_seq, int verify,
+                                                        int dh, double log2_base,
+                                                        __nv_bfloat16* __restrict__ xq,
+                                                        float2* __restrict__ rope_tab) {
+  grid_dep_launch();
+  const int m = blockIdx.x;
+  const int ps = idx[m];
+  const bool ok = ps >= 0 && ps < N;
+  if (!verify) {
+    const int b = m / rows_per_seq;
+    const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)b * N + (ok ? ps : 0)) * D);
+    uint4* dst = reinterpret_cast<uint4*>(xq + (size_t)m * D);
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = threadIdx.x; i < D / 8; i += blockDim.x) dst[i] = ok ? __ldg(src + i) : zero;
+  }
+  const int half = dh / 2;
+  for (int j = threadIdx.x; j < half; j += blockDim.x) {
+    float c, s;
+    rope_cos_sin(ok ? ps : 0, rope_inv_freq(j, dh, log2_base), &c, &s);
+    rope_tab[(size_t)m * half + j] = make_float2(c, s);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+               ProjTcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int BN = p.BN;
+  const uint32_t bsub_bytes = (uint32_t)BN * 128u;
+  const uint32_t stage_bytes = (uint32_t)p.subs * (kASubBytes + bsub_bytes);
+  float* staging = reinterpret_cast<float*>(smem + p.nstage * stage_bytes);
+  uint8_t* misc = reinterpret_cast<uint8_t*>(staging + kBM * kPitch);
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc);
+  uint64_t* empty = full + p.nstage;
+  uint64_t* acc_full = empty + p.nstage;   // [2]
+  uint64_t* acc_empty = acc_full + 2;      // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* last_flag = abort_flag + 1;
+  int* tok_slot = reinterpret_cast<int*>(misc + 256);  // -1: skip k, v
+  int* tok_flag = tok_slot + kMaxBN;                   // bit0: q valid, bit1: side buffer
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int G = gridDim.x, c = blockIdx.x;
+  const long long u_begin = unit_lo(p.total_units, G, c);
+  const long long u_end = unit_lo(p.total_units, G, c + 1);
+
+  uint32_t ncols = 32;
+  while ((int)ncols < 2 * BN) ncols <<= 1;
+
+  if (tid == 0) {
+    for (int s = 0; s < p.nstage; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&acc_full[b], 1);
+      tc::mbar_init(&acc_empty[b], kEpiThreads);
+    }
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc(tmem_slot, ncols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_w);
+      tc::prefetch_tmap(&tm_x);
+      const uint64_t pol_w = p.n_tt > 1 ? tc::policy_evict_normal() : tc::policy_evict_first();
+      const uint64_t pol_x = tc::policy_evict_last();
+      const long long n_units = u_end - u_begin;
+      // W does not depend on the prep kernel: fill the first stages before
+      // waiting for it, then add their X boxes.
+      const int pre = (int)(n_units < p.nstage ? n_units : p.nstage);
+      for (int i = 0; i < pre; ++i) {
+        const long long u = u_begin + i;
+        const int tile = (int)(u / p.nks), ks = (int)(u % p.nks);
+        const int sb0 = ks * p.subs, nsub = min(p.subs, p.nsub_total - sb0);
+        uint8_t* a_s = smem + i * stage_bytes;
+        tc::mbar_arrive_expect_tx(&full[i], (uint32_t)nsub * (kASubBytes + bsub_bytes));
+        for (int q = 0; q < nsub; ++q)
+          tc::tma_load_2d(a_s + q * kASubBytes, &tm_w, &full[i], (sb0 + q) * kSub,
+                          (tile / p.n_tt) * kBM, pol_w);
+      }
+      grid_dep_wait();
+      for (int i = 0; i < pre; ++i) {
+        const long long u = u_begin + i;
+        const int tile = (int)(u / p.nks), ks = (int)(u % p.nks);
+        const int sb0 = ks * p.subs, nsub = min(p.subs, p.nsub_total - sb0);
+        uint8_t* b_s = smem + i * stage_bytes + p.subs * kASubBytes;
+        for (int q = 0; q < nsub; ++q)
+          tc::tma_load_2d(b_s + q * bsub_bytes, &tm_x, &full[i], (sb0 + q) * kSub,
+                          (tile % p.n_tt) * BN, pol_x);
+      }
+      for (long long u = u_begin + pre; u < u_end; ++u) {
+        const int it = (int)(u - u_begin);
+        const int s = it % p.nstage;
+        const uint32_t ph = (uint32_t)(it / p.nstage) & 1u;
+        if (!tc::mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status)) break;
+        const int tile = (int)(u / p.nks), ks = (int)(u % p.nks);
+        const int sb0 = ks * p.subs, nsub = min(p.subs, p.nsub_total - sb0);
+        uint8_t* a_s = smem + s * stage_bytes;
+        uint8_t* b_s = a_s + p.subs * kASubBytes;
+        // rows of X past M are outside the tensor: TMA fills them with zeros
+        tc::mbar_arrive_expect_tx(&full[s], (uint32_t)nsub * (kASubBytes + bsub_bytes));
+        for (int q = 0; q < nsub; ++q) {
+          tc::tma_load_2d(a_s + q * kASubBytes, &tm_w, &full[s], (sb0 + q) * kSub,
+                          (tile / p.n_tt) * kBM, pol_w);
+          tc::tma_load_2d(b_s + q * bsub_bytes, &tm_x, &full[s], (sb0 + q) * kSub,
+                          (tile % p.n_tt) * BN, pol_x);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16(kBM, BN);
+      int it = 0, j = 0;
+      bool ok = true;
+      for (long long u = u_begin; u < u_end && ok; ++j) {
+        const int ks0 = (int)(u % p.nks);
+        const int ks1 = (int)min((long long)p.nks, ks0 + (u_end - u));
+        u += ks1 - ks0;
+        const int buf = j & 1;
+        if (!tc::mbar_wait(&acc_empty[buf], ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, p.status)) break;
+        tc::tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(buf * BN);
+        for (int ks = ks0; ks < ks1; ++ks, ++it) {
+          const int s = it % p.nstage;
+          const uint32_t ph = (uint32_t)(it / p.nstage) & 1u;
+          if (!tc::mbar_wait(&full[s], ph, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const int nsub = min(p.subs, p.nsub_total - ks * p.subs);
+          const uint32_t a_addr = tc::smem_u32(smem + s * stage_bytes);
+          const uint32_t b_addr = a_addr + p.subs * kASubBytes;
+          for (int q = 0; q < nsub; ++q) {
+#pragma unroll
+            for (int kk = 0; kk < kSub / 16; ++kk) {
+              const uint64_t da = tc::smem_desc(a_addr + q * kASubBytes + kk * 32, 16, 1024, 2);
+              const uint64_t db = tc::smem_desc(b_addr + q * bsub_bytes + kk * 32, 16, 1024, 2);
+              tc::mma_bf16(d_tmem, da, db, idesc, (ks != ks0 || q != 0 || kk != 0) ? 1u : 0u);
+            }
+          }
+          tc::mma_commit(&empty[s]);
+        }
+        tc::mma_commit(&acc_full[buf]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    grid_dep_wait();  // the RoPE table comes from the prep kernel
+    const int etid = tid - 64;
+    const int quarter = warp & 3;
+    const int f_loc = quarter * 32 + lane;
+    const int half = p.dh >> 1;
+    float* my_parts = p.partials + (size_t)c * 2 * BN * kBM;
+    int j = 0;
+    for (long long u = u_begin; u < u_end; ++j) {
+      const int tile = (int)(u / p.nks);
+      const int ks0 = (int)(u % p.nks);
+      const int ks1 = (int)min((long long)p.nks, ks0 + (u_end - u));
+      u += ks1 - ks0;
+      const int buf = j & 1;
+      const int ft = tile / p.n_tt, tt = tile % p.n_tt;
+      const int m0 = tt * BN;
+      const bool whole = (ks0 == 0 && ks1 == p.nks);
+      const uint32_t t_acc = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
+
+      // token routing of this tile, ahead of the accumulator
+      for (int n = etid; n < BN; n += kEpiThreads) {
+        const int m = m0 + n;
+        int slot = -1, flag = 0;
+        if (m < p.M) {
+          const int ps = p.idx[m];
+          const bool in_range = ps >= 0 && ps < p.N;
+          if (in_range) flag |= 1;
+          if (p.verify && p.view[m] == 2) {
+            int s = 0;
+            const int b = m / p.rows_per_seq;
+            for (int r = b * p.rows_per_seq; r < m; ++r) s += (p.view[r] == 2);
+            flag |= 2;
+            slot = (in_range && s < p.S_max) ? s : -1;
+          } else {
+            slot = in_range ? ps : -1;
+          }
+        }
+        tok_slot[n] = slot;
+        tok_flag[n] = flag;
+      }
+
+      if (!tc::mbar_wait(&acc_full[buf], (uint32_t)(j >> 1) & 1u, abort_flag, p.status)) break;
+      tc::tc_fence_after();
+
+      bool run = true;
+      int c_first = c, c_last = c;
+      if (!whole) {
+        // partial tile: store it, free the accumulator, and see who is last
+        const int slot = (tile == (int)(u_begin / p.nks)) ? 0 : 1;
+        float* dst = my_parts + (size_t)slot * BN * kBM;
+        for (int cc = 0; cc < BN; cc += kChunk) {
+          float v[kChunk];
+          tc::tmem_ld32(t_acc + cc, v);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int n = 0; n < kChunk; ++n)
+            if (cc + n < BN) dst[(size_t)(cc + n) * kBM + f_loc] = v[n];
+        }
+        tc::tc_fence_before();
+        tc::mbar_arrive(&acc_empty[buf]);
+        __threadfence();
+        const long long tu0 = (long long)tile * p.nks;
+        c_first = owner_of(tu0, p.total_units, G);
+        c_last = owner_of(tu0 + p.nks - 1, p.total_units, G);
+        tc::named_bar_sync(1, kEpiThreads);
+        if (etid == 0) {
+          const unsigned prev = atomicAdd(&p.tile_cnt[tile], 1u);
+          *last_flag = (prev == (unsigned)(c_last - c_first));
+          if (*last_flag) p.tile_cnt[tile] = 0u;
+        }
+        tc::named_bar_sync(1, kEpiThreads);
+        run = *last_flag != 0;
+        if (run) __threadfence();
+      }
+      if (run) {
+        if (ft == 0) {
+          for (int n = etid; n < BN; n += kEpiThreads)
+            if (m0 + n < p.M && tok_slot[n] < 0) set_status(p.status, FDLLM_ERR_BAD_INDEX);
+        }
+        for (int cc = 0; cc < BN; cc += kChunk) {
+          if (whole) {
+            float v[kChunk];
+            tc::tmem_ld32(t_acc + cc, v);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int n = 0; n < kChunk; ++n) staging[f_loc * kPitch + n] = v[n];
+          } else {
+            // sum the partials of every contributor in k order; a thread adds
+            // 4 consecutive features of 8 tokens with 16-byte loads
+            float4 acc[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            const int f4 = (etid & 31) * 4;
+            const int nb = etid >> 5;  // tokens nb, nb + 4, ...
+            for (int cb = c_first; cb <= c_last; ++cb) {
+              const int sl = (tile == (int)(unit_lo(p.total_units, G, cb) / p.nks)) ? 0 : 1;
+              const float* ps = p.partials + ((size_t)cb * 2 + sl) * BN * kBM;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const int n = cc + nb + 4 * i;
+                if (n < BN) {
+                  const float4 t = __ldcg(reinterpret_cast<const float4*>(ps + (size_t)n * kBM + f4));
+                  acc[i].x += t.x; acc[i].y += t.y; acc[i].z += t.z; acc[i].w += t.w;
+                }
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int n = nb + 4 * i;
+              staging[(f4 + 0) * kPitch + n] = acc[i].x;
+              staging[(f4 + 1) * kPitch + n] = acc[i].y;
+              staging[(f4 + 2) * kPitch + n] = acc[i].z;
+              staging[(f4 + 3) * kPitch + n] = acc[i].w;
+            }
+          }
+          tc::named_bar_sync(1, kEpiThreads);
+          // 32 tokens x 16 groups of 8 features; a warp covers 32 tokens of one group
+          for (int itm = etid; itm < kChunk * (kBM / 8); itm += kEpiThreads) {
+            const int g = itm / kChunk, n = itm % kChunk;
+            const int m = m0 + cc + n;
+            if (cc + n >= BN || m >= p.M) continue;
+            const int f0 = g * 8;
+            const int fg = ft * kBM + f0;
+            if (fg >= p.F) continue;
+            const int blk = fg / p.E, rem = fg % p.E;
+            const int h = rem / p.dh, j0 = rem % p.dh;
+            const int slot = tok_slot[cc + n], flag = tok_flag[cc + n];
+            if (blk != 0 && slot < 0) continue;
+            float o[8];
+            if (blk == 2) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) o[i] = staging[(f0 + i) * kPitch + n];
+            } else if (blk == 0 && !(flag & 1)) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) o[i] = 0.f;  // a skipped query attends with q = 0
+            } else {
+              const bool lo = j0 < half;
+              const int pf = lo ? f0 + half : f0 - half;
+              const float2* tab = p.rope_tab + (size_t)m * half + (lo ? j0 : j0 - half);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float x = staging[(f0 + i) * kPitch + n];
+                const float xp = staging[(pf + i) * kPitch + n];
+                const float2 cs = __ldg(tab + i);
+                o[i] = lo ? (x * cs.x - xp * cs.y) : (xp * cs.y + x * cs.x);
+              }
+            }
+            uint4 pk;
+            pk.x = pack_bf16x2(o[0], o[1]);
+            pk.y = pack_bf16x2(o[2], o[3]);
+            pk.z = pack_bf16x2(o[4], o[5]);
+            pk.w = pack_bf16x2(o[6], o[7]);
+            __nv_bfloat16* dst;
+            if (blk == 0) {
+              dst = p.q_out + (size_t)m * p.E + h * p.dh + j0;
+            } else {
+              const bool side = (flag & 2) != 0;
+              __nv_bfloat16* base = (blk == 1) ? (side ? p.k_side : p.k_cache)
+                                               : (side ? p.v_side : p.v_cache);
+              const int nslots = side ? p.S_max : p.N;
+              const int b = m / p.rows_per_seq;
+              dst = base + (((size_t)b * p.H + h) * nslots + slot) * p.dh + j0;
+            }
+            *reinterpret_cast<uint4*>(dst) = pk;
+          }
+          tc::named_bar_sync(1, kEpiThreads);
+        }
+      }
+      if (whole) {
+        tc::tc_fence_before();
+        tc::mbar_arrive(&acc_empty[buf]);
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tc::tmem_dealloc(tmem, ncols);
+  }
+}
+
+struct ProjPlan {
+  int BN, n_tt, n_ft, tiles, nks, subs, nsub_total, nstage, grid;
+  long long total_units;
+  size_t smem_bytes, partial_bytes, counter_bytes, xq_bytes, tab_bytes;
+};
+
+constexpr size_t kSmemBudget = 227 * 1024;
+
+ProjPlan plan(int M, int D, int H, int dh, int num_sms) {
+  ProjPlan q{};
+  const int F = 3 * H * dh;
+  q.n_tt = (M + kMaxBN - 1) / kMaxBN;
+  const int per = (M + q.n_tt - 1) / q.n_tt;
+  q.BN = ((per + 15) / 16) * 16;
+  q.n_ft = (F + kBM - 1) / kBM;
+  q.tiles = q.n_ft * q.n_tt;
+  q.nsub_total = D / kSub;
+  const size_t fixed = 1024 /*align*/ + (size_t)kBM * kPitch * 4 + 256 + 2 * kMaxBN * 4;
+  // the widest k-step (most contiguous bytes per W row) that keeps two stages
+  const int cand[3] = {4, 2, 1};
+  for (int i = 0; i < 3; ++i) {
+    const int subs = cand[i];
+    const size_t stage = (size_t)subs * (kASubBytes + (size_t)q.BN * 128);
+    const int ns = (int)((kSmemBudget - fixed) / stage);
+    if (ns >= 2 || subs == 1) {
+      q.subs = subs;
+      q.nstage = ns < 8 ? ns : 8;
+      break;
+    }
+  }
+  if (q.subs > q.nsub_total) q.subs = q.nsub_total;
+  const size_t stage = (size_t)q.subs * (kASubBytes + (size_t)q.BN * 128);
+  if ((int)((kSmemBudget - fixed) / stage) < q.nstage) q.nstage = (int)((kSmemBudget - fixed) / stage);
+  q.nks = (q.nsub_total + q.subs - 1) / q.subs;
+  q.total_units = (long long)q.tiles * q.nks;
+  q.grid = (int)(q.total_units < num_sms ? q.total_units : num_sms);
+  q.smem_bytes = (size_t)q.nstage * stage + fixed;
+  q.partial_bytes = align_up((size_t)q.grid * 2 * q.BN * kBM * sizeof(float), 256);
+  q.counter_bytes = align_up((size_t)q.tiles * sizeof(unsigned), 256);
+  q.xq_bytes = align_up((size_t)M * D * 2, 256);
+  q.tab_bytes = align_up((size_t)M * (dh / 2) * sizeof(float2), 256);
+  return q;
+}
+
+}  // namespace
+
+size_t proj_tc_workspace_bytes(int M, int D, int H, int dh, int num_sms) {
+  if (M <= 0) return 256;
+  const ProjPlan q = plan(M, D, H, dh, num_sms);
+  return q.partial_bytes + q.counter_bytes + q.xq_bytes + q.tab_bytes;
+}
+
+cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream) {
+  const int M = a.B * a.rows_per_seq;
+  if (M == 0) return cudaSuccess;
+  const int E = a.H * a.dh, F = 3 * E;
+  const ProjPlan q = plan(M, a.D, a.H, a.dh, device_sm_count());
+  if (q.partial_bytes + q.counter_bytes + q.xq_bytes + q.tab_bytes > a.ws_bytes)
+    return cudaErrorInvalidValue;
+  char* ws = static_cast<char*>(a.ws);
+  __nv_bfloat16* xq = reinterpret_cast<__nv_bfloat16*>(ws + q.partial_bytes + q.counter_bytes);
+  float2* tab = reinterpret_cast<float2*>(ws + q.partial_bytes + q.counter_bytes + q.xq_bytes);
+
+  CUtensorMap tm_w, tm_x;
+  {
+    const uint64_t dims[2] = {(uint64_t)a.D, (uint64_t)F};
+    const uint64_t strides[1] = {(uint64_t)a.D * 2};
+    const uint32_t box[2] = {kSub, kBM};
+    if (!encode_bf16_map(&tm_w, 2, a.w, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+      return cudaErrorInvalidValue;
+  }
+  // X: the packed verify rows, or x[Q] packed into the workspace by the prep kernel
+  const void* xsrc = a.verify ? a.x : static_cast<const void*>(xq);
+  {
+    const uint64_t dims[2] = {(uint64_t)a.D, (uint64_t)M};
+    const uint64_t strides[1] = {(uint64_t)a.D * 2};
+    const uint32_t box[2] = {kSub, (uint32_t)q.BN};
+    if (!encode_bf16_map(&tm_x, 2, xsrc, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
+      return cudaErrorInvalidValue;
+  }
+  ProjTcParams p{};
+  p.M = M; p.F = F; p.D = a.D; p.E = E; p.N = a.N; p.H = a.H; p.dh = a.dh;
+  p.rows_per_seq = a.rows_per_seq; p.S_max = a.S_max; p.verify = a.verify;
+  p.BN = q.BN; p.n_tt = q.n_tt; p.tiles = q.tiles; p.nks = q.nks; p.subs = q.subs;
+  p.nsub_total = q.nsub_total; p.nstage = q.nstage; p.total_units = q.total_units;
+  p.idx = a.idx; p.view = a.view; p.rope_tab = tab;
+  p.k_cache = static_cast<__nv_bfloat16*>(a.k_cache);
+  p.v_cache = static_cast<__nv_bfloat16*>(a.v_cache);
+  p.k_side = static_cast<__nv_bfloat16*>(a.k_side);
+  p.v_side = static_cast<__nv_bfloat16*>(a.v_side);
+  p.q_out = static_cast<__nv_bfloat16*>(a.q_out);
+  p.status = a.status;
+  p.partials = reinterpret_cast<float*>(ws);
+  p.tile_cnt = reinterpret_cast<unsigned*>(ws + q.partial_bytes);
+
+  proj_prep_kernel<<<M, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.x), a.idx, a.N,
+                                          a.D, a.rows_per_seq, a.verify, a.dh, a.log2_base, xq,
+                                          tab);
+  count_launches(1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  e = cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)q.smem_bytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(q.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = q.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, proj_tc_kernel, tm_w, tm_x, p);
+  count_launches(1);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace fdllm
