@@ -13,7 +13,7 @@ using namespace fdllm;
 namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
-constexpr int kMaxVerifyRows = 4000;
+constexpr int kMaxVerifyRows = 512;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

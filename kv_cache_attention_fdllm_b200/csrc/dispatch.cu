@@ -16,12 +16,13 @@ cudaError_t launch_proj(const ProjArgs& a, cudaStream_t stream) {
 
 size_t attn_workspace_bytes(int B, int N, int H, int dh, int rows_per_seq, int S_max, int verify,
                             int dtype, int num_sms) {
-  (void)B; (void)N; (void)H; (void)dh; (void)rows_per_seq; (void)S_max; (void)verify;
-  (void)dtype; (void)num_sms;
+  if (dtype == FDLLM_BF16)
+    return attn_tc_workspace_bytes(B, N, H, dh, rows_per_seq, S_max, verify, num_sms);
   return 0;
 }
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream) {
+  if (a.dtype == FDLLM_BF16) return launch_attn_tc(a, stream);
   return launch_attn_simt(a, stream);
 }
 

@@ -86,6 +86,9 @@ size_t proj_tc_workspace_bytes(int M, int D, int H, int dh, int num_sms);
 cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream);
 cudaError_t launch_proj_simt(const ProjArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t stream);
+size_t attn_tc_workspace_bytes(int B, int N, int H, int dh, int rows, int S_max, int verify,
+                               int num_sms);
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream);
 
 // ----------------------------------------------------------------- helpers
 int device_sm_count();

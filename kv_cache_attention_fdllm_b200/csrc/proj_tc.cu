@@ -296,7 +296,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         tok_flag[n] = flag;
       }
 
-      if (!tc::mbar_wait(&acc_full[buf], (uint32_t)(j >> 1) & 1u, abort_flag, p.status)) break;
+      // after a timeout every later wait returns at once: keep going so that all
+      // epilogue threads still meet at the same named barriers
+      tc::mbar_wait(&acc_full[buf], (uint32_t)(j >> 1) & 1u, abort_flag, p.status);
       tc::tc_fence_after();
 
       bool run = true;
