@@ -35,15 +35,13 @@ namespace fdllm {
 namespace {
 
 constexpr int kKT = 128;  // keys per tile
-constexpr int kThreads = 192;
-constexpr int kSmx = 128;  // softmax threads
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kThresh = 8.f;  // lazy rescale threshold (log2 units)
 constexpr int kMaxRows = 512;   // verify rows per sequence held in shared memory
 
 struct AttnTcParams {
   int B, N, H, rows, S_max, causal;
-  int n_qc, n_cache_tiles, n_side_tiles, tpi, nstage;
+  int n_qc, n_cache_tiles, n_side_tiles, tpi, nk, nv;
   long long total_units;
   float qk_scale;  // log2(e) / sqrt(dh)
   const int32_t* pos;
@@ -85,6 +83,34 @@ __device__ __forceinline__ bool bar_any(int id, int n, bool pred) {
   return r != 0;
 }
 
+// Bookkeeping for polling loops: after kWaitLimitNs without progress the
+// loop gives up (records FDLLM_ERR_TIMEOUT and sets the abort flag).
+struct IdleClock {
+  uint64_t t0 = 0;
+  uint32_t spins = 0;
+  __device__ __forceinline__ void reset() { t0 = 0; spins = 0; }
+  __device__ __forceinline__ bool idle(volatile int* abort, int* status) {
+    if ((++spins & 63u) != 0) return true;
+    if (*abort) return false;
+    const uint64_t now = global_ns();
+    if (t0 == 0) {
+      t0 = now;
+    } else if (now - t0 > kWaitLimitNs) {
+      *abort = 1;
+      set_status(status, FDLLM_ERR_TIMEOUT);
+      return false;
+    }
+    return true;
+  }
+};
+
+// 2^x on the special-function unit (flush-to-zero; 2^-inf = 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int NQ>
 __device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float* v) {
 #pragma unroll
@@ -101,34 +127,47 @@ template <int NQ, int DH>
 struct Smem {
   static constexpr int kBoxes = DH / 64;
   static constexpr uint32_t kTileBytes = kBoxes * 16384;         // K or V tile
-  static constexpr uint32_t kStageBytes = 2 * kTileBytes;        // K then V
   static constexpr uint32_t kQBytes = kBoxes * NQ * 128;         // one Q chunk
   static constexpr uint32_t kPRow = NQ * 2;                      // bytes per key row of P
   static constexpr uint32_t kPBytes = kKT * kPRow;
+  static constexpr uint32_t kPBufBytes = (kPBytes + 1023) / 1024 * 1024;  // one of two P buffers
+};
+
+// Softmax threads: NQ/16 groups of 4 warps; a thread owns one key (one dh row)
+// and 16 query columns.
+template <int NQ>
+struct Threads {
+  static constexpr int kSmx = 8 * NQ;
+  static constexpr int kAll = 64 + kSmx;
 };
 
 template <int NQ, int DH, bool VERIFY>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Threads<NQ>::kAll, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_ks,
                const __grid_constant__ CUtensorMap tm_vs, AttnTcParams p) {
   using L = Smem<NQ, DH>;
+  constexpr int kSmx = Threads<NQ>::kSmx;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const int NS = p.nstage;
-  uint8_t* q_buf = smem + NS * L::kStageBytes;
+  const int NK = p.nk, NV = p.nv;
+  uint8_t* k_ring = smem;
+  uint8_t* v_ring = smem + NK * L::kTileBytes;
+  uint8_t* q_buf = v_ring + NV * L::kTileBytes;
   uint8_t* p_buf = q_buf + 2 * L::kQBytes;  // 1024-aligned (kQBytes is a multiple of 1024)
-  uint8_t* misc = p_buf + ((L::kPBytes + 1023) / 1024) * 1024;
-  uint64_t* kv_full = reinterpret_cast<uint64_t*>(misc);
-  uint64_t* kv_empty = kv_full + 8;
-  uint64_t* q_full = kv_empty + 8;   // [2]
+  uint8_t* misc = p_buf + 2 * L::kPBufBytes;
+  uint64_t* k_full = reinterpret_cast<uint64_t*>(misc);
+  uint64_t* k_empty = k_full + 8;
+  uint64_t* v_full = k_empty + 8;
+  uint64_t* v_empty = v_full + 8;
+  uint64_t* q_full = v_empty + 8;    // [2]
   uint64_t* q_empty = q_full + 2;    // [2]
   uint64_t* s_full = q_empty + 2;    // [2]
   uint64_t* s_empty = s_full + 2;    // [2]
-  uint64_t* p_full = s_empty + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 1);
+  uint64_t* p_full = s_empty + 2;    // [2]
+  uint64_t* pv_done = p_full + 2;    // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* last_flag = abort_flag + 1;
   int* n_draft_s = last_flag + 1;
@@ -153,18 +192,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   while ((int)ncols < 3 * NQ) ncols <<= 1;
 
   if (tid == 0) {
-    for (int s = 0; s < NS; ++s) {
-      tc::mbar_init(&kv_full[s], 1);
-      tc::mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < NK; ++s) {
+      tc::mbar_init(&k_full[s], 1);
+      tc::mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      tc::mbar_init(&v_full[s], 1);
+      tc::mbar_init(&v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&q_full[b], 1);
       tc::mbar_init(&q_empty[b], 1);
       tc::mbar_init(&s_full[b], 1);
-      tc::mbar_init(&s_empty[b], kSmx);
+      tc::mbar_init(&s_empty[b], kSmx / 32);  // one arrival per softmax warp
     }
-    tc::mbar_init(p_full, kSmx);
-    tc::mbar_init(pv_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&p_full[b], kSmx / 32);
+      tc::mbar_init(&pv_done[b], 1);
+    }
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -177,104 +222,150 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // K and V have their own rings; each is filled as soon as its stage frees
+    // (a K stage right after its QK, a V stage after its PV), polling both so
+    // that neither stream waits behind the other.
     if (lane == 0) {
       tc::prefetch_tmap(&tm_q);
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
       const uint64_t pol_kv = tc::policy_evict_first();
       const uint64_t pol_q = tc::policy_evict_last();
-      int seg = -1;
-      for (int i = 0; i < T; ++i) {
-        const long long u = u0 + i;
-        const int item = (int)(u / tpi), t = (int)(u % tpi);
-        const int qc = item % p.n_qc, bh = item / p.n_qc;
-        const int b = bh / p.H, h = bh % p.H;
-        if (i == 0 || t == 0) {
-          ++seg;
-          const int qb = seg & 1;
-          if (!tc::mbar_wait(&q_empty[qb], ((uint32_t)(seg >> 1) & 1u) ^ 1u, abort_flag, p.status)) break;
-          tc::mbar_arrive_expect_tx(&q_full[qb], L::kQBytes);
+      int ik = 0, iv = 0, seg = -1;
+      IdleClock clk;
+      while (iv < T) {
+        bool progressed = false;
+        if (ik < T) {
+          const long long u = u0 + ik;
+          const int item = (int)(u / tpi), t = (int)(u % tpi);
+          const int qc = item % p.n_qc, bh = item / p.n_qc;
+          const bool first = (ik == 0 || t == 0);
+          const int qb = (seg + 1) & 1;
+          const int ks = ik % NK;
+          if (tc::mbar_test(&k_empty[ks], ((uint32_t)(ik / NK) & 1u) ^ 1u) &&
+              (!first || tc::mbar_test(&q_empty[qb], ((uint32_t)((seg + 1) >> 1) & 1u) ^ 1u))) {
+            if (first) {
+              ++seg;
+              tc::mbar_arrive_expect_tx(&q_full[qb], L::kQBytes);
 #pragma unroll
-          for (int x = 0; x < L::kBoxes; ++x)
-            tc::tma_load_4d(q_buf + qb * L::kQBytes + x * NQ * 128, &tm_q, &q_full[qb], x * 64, h,
-                            qc * NQ, b, pol_q);
-        }
-        const int s = i % NS;
-        if (!tc::mbar_wait(&kv_empty[s], ((uint32_t)(i / NS) & 1u) ^ 1u, abort_flag, p.status)) break;
-        uint8_t* kd = smem + s * L::kStageBytes;
-        uint8_t* vd = kd + L::kTileBytes;
-        tc::mbar_arrive_expect_tx(&kv_full[s], L::kStageBytes);
-        const bool side = VERIFY && t >= p.n_cache_tiles;
-        const int key0 = (side ? t - p.n_cache_tiles : t) * kKT;
+              for (int x = 0; x < L::kBoxes; ++x)
+                tc::tma_load_4d(q_buf + qb * L::kQBytes + x * NQ * 128, &tm_q, &q_full[qb], x * 64,
+                                bh % p.H, qc * NQ, bh / p.H, pol_q);
+            }
+            const bool side = VERIFY && t >= p.n_cache_tiles;
+            const int key0 = (side ? t - p.n_cache_tiles : t) * kKT;
+            uint8_t* kd = k_ring + ks * L::kTileBytes;
+            tc::mbar_arrive_expect_tx(&k_full[ks], L::kTileBytes);
 #pragma unroll
-        for (int x = 0; x < L::kBoxes; ++x) {
-          tc::tma_load_3d(kd + x * 16384, side ? &tm_ks : &tm_k, &kv_full[s], x * 64, key0, bh, pol_kv);
-          tc::tma_load_3d(vd + x * 16384, side ? &tm_vs : &tm_v, &kv_full[s], x * 64, key0, bh, pol_kv);
+            for (int x = 0; x < L::kBoxes; ++x)
+              tc::tma_load_3d(kd + x * 16384, side ? &tm_ks : &tm_k, &k_full[ks], x * 64, key0, bh, pol_kv);
+            ++ik;
+            progressed = true;
+          }
         }
+        if (iv < ik) {
+          const int vs = iv % NV;
+          if (tc::mbar_test(&v_empty[vs], ((uint32_t)(iv / NV) & 1u) ^ 1u)) {
+            const long long u = u0 + iv;
+            const int item = (int)(u / tpi), t = (int)(u % tpi);
+            const int bh = item / p.n_qc;
+            const bool side = VERIFY && t >= p.n_cache_tiles;
+            const int key0 = (side ? t - p.n_cache_tiles : t) * kKT;
+            uint8_t* vd = v_ring + vs * L::kTileBytes;
+            tc::mbar_arrive_expect_tx(&v_full[vs], L::kTileBytes);
+#pragma unroll
+            for (int x = 0; x < L::kBoxes; ++x)
+              tc::tma_load_3d(vd + x * 16384, side ? &tm_vs : &tm_v, &v_full[vs], x * 64, key0, bh, pol_kv);
+            ++iv;
+            progressed = true;
+          }
+        }
+        if (!progressed && !clk.idle(abort_flag, p.status)) break;
+        if (progressed) clk.reset();
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Two in-order streams, QK(i) and PV(j), each issued as soon as its inputs
+    // are ready, so neither waits behind the other.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = tc::idesc_bf16(kKT, NQ, false, false);
       constexpr uint32_t idesc_pv = tc::idesc_bf16(kKT, NQ, true, true);
       constexpr uint32_t p_swz = NQ == 64 ? 2u : (NQ == 32 ? 4u : 6u);
       const uint32_t p_addr = tc::smem_u32(p_buf);
-      int seg = -1;
-      bool ok = true;
-      for (int i = 0; i <= T && ok; ++i) {
-        if (i < T) {
-          const long long u = u0 + i;
+      int iq = 0, ip = 0, seg = -1;
+      IdleClock clk;
+      while (ip < T) {
+        bool progressed = false;
+        if (iq < T) {
+          const long long u = u0 + iq;
           const int t = (int)(u % tpi);
-          const bool first = (i == 0 || t == 0);
-          const bool last = (i == T - 1 || t == tpi - 1);
-          if (first) ++seg;
-          const int qb = seg & 1;
-          const int s = i % NS;
-          if (!tc::mbar_wait(&kv_full[s], (uint32_t)(i / NS) & 1u, abort_flag, p.status)) { ok = false; break; }
-          if (first && !tc::mbar_wait(&q_full[qb], (uint32_t)(seg >> 1) & 1u, abort_flag, p.status)) { ok = false; break; }
-          const int sb = i & 1;
-          if (!tc::mbar_wait(&s_empty[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
-          tc::tc_fence_after();
-          const uint32_t k_addr = tc::smem_u32(smem + s * L::kStageBytes);
-          const uint32_t q_addr = tc::smem_u32(q_buf + qb * L::kQBytes);
+          const bool first = (iq == 0 || t == 0);
+          const bool last = (iq == T - 1 || t == tpi - 1);
+          const int qb = first ? ((seg + 1) & 1) : (seg & 1);
+          const int qseg = first ? seg + 1 : seg;
+          const int ks = iq % NK, sb = iq & 1;
+          if (tc::mbar_test(&k_full[ks], (uint32_t)(iq / NK) & 1u) &&
+              tc::mbar_test(&s_empty[sb], ((uint32_t)(iq >> 1) & 1u) ^ 1u) &&
+              (!first || tc::mbar_test(&q_full[qb], (uint32_t)(qseg >> 1) & 1u))) {
+            seg = qseg;
+            tc::tc_fence_after();
+            const uint32_t k_addr = tc::smem_u32(k_ring + ks * L::kTileBytes);
+            const uint32_t q_addr = tc::smem_u32(q_buf + qb * L::kQBytes);
 #pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk) {
-            const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t qo = (kk >> 2) * NQ * 128 + (kk & 3) * 32;
-            tc::mma_bf16(tmem + sb * NQ, tc::smem_desc(k_addr + ko, 16, 1024, 2),
-                         tc::smem_desc(q_addr + qo, 16, 1024, 2), idesc_qk, kk != 0);
+            for (int kk = 0; kk < DH / 16; ++kk) {
+              const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
+              const uint32_t qo = (kk >> 2) * NQ * 128 + (kk & 3) * 32;
+              tc::mma_bf16(tmem + sb * NQ, tc::smem_desc(k_addr + ko, 16, 1024, 2),
+                           tc::smem_desc(q_addr + qo, 16, 1024, 2), idesc_qk, kk != 0);
+            }
+            tc::mma_commit(&s_full[sb]);
+            tc::mma_commit(&k_empty[ks]);
+            if (last) tc::mma_commit(&q_empty[qb]);
+            ++iq;
+            progressed = true;
           }
-          tc::mma_commit(&s_full[sb]);
-          if (last) tc::mma_commit(&q_empty[qb]);
         }
-        if (i >= 1) {
-          const int j = i - 1;
-          const long long u = u0 + j;
-          const bool first = (j == 0 || (u % tpi) == 0);
-          if (!tc::mbar_wait(p_full, (uint32_t)j & 1u, abort_flag, p.status)) { ok = false; break; }
-          tc::tc_fence_after();
-          const int s = j % NS;
-          const uint32_t v_addr = tc::smem_u32(smem + s * L::kStageBytes + L::kTileBytes);
+        if (ip < iq) {
+          const int vs = ip % NV;
+          if (tc::mbar_test(&p_full[ip & 1], (uint32_t)(ip >> 1) & 1u) &&
+              tc::mbar_test(&v_full[vs], (uint32_t)(ip / NV) & 1u)) {
+            const long long u = u0 + ip;
+            const bool first = (ip == 0 || (u % tpi) == 0);
+            tc::tc_fence_after();
+            const uint32_t v_addr = tc::smem_u32(v_ring + vs * L::kTileBytes);
+            const uint32_t pb_addr = p_addr + (ip & 1) * L::kPBufBytes;
 #pragma unroll
-          for (int kk = 0; kk < kKT / 16; ++kk) {
-            const uint64_t da = tc::smem_desc(v_addr + kk * 2048, DH == 128 ? 16384 : 0, 1024, 2);
-            const uint64_t db = tc::smem_desc(p_addr + kk * 16 * L::kPRow, 0, 8 * L::kPRow, p_swz);
-            tc::mma_bf16(tmem_o, da, db, idesc_pv, (first && kk == 0) ? 0u : 1u);
+            for (int kk = 0; kk < kKT / 16; ++kk) {
+              const uint64_t da = tc::smem_desc(v_addr + kk * 2048, DH == 128 ? 16384 : 0, 1024, 2);
+              const uint64_t db = tc::smem_desc(pb_addr + kk * 16 * L::kPRow, 0, 8 * L::kPRow, p_swz);
+              tc::mma_bf16(tmem_o, da, db, idesc_pv, (first && kk == 0) ? 0u : 1u);
+            }
+            tc::mma_commit(&pv_done[ip & 1]);
+            tc::mma_commit(&v_empty[vs]);
+            ++ip;
+            progressed = true;
           }
-          tc::mma_commit(pv_done);
-          tc::mma_commit(&kv_empty[s]);
         }
+        if (!progressed && !clk.idle(abort_flag, p.status)) break;
+        if (progressed) clk.reset();
       }
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int st = tid - 64;           // 0..127
+    // NQ/16 groups of 4 warps: the warps that share a TMEM lane quarter split
+    // the query columns, so a thread owns one key (later one dh row) and the
+    // 16 columns [c0, c0 + 16).
+    constexpr int NQH = 16;
+    const int st = tid - 64;                 // 0..kSmx-1
     const int quarter = warp & 3;
-    const int kl = quarter * 32 + lane;  // TMEM lane: key of S^T, dh row of O^T
+    const int half = (warp - 2) >> 2;        // column group
+    const int c0 = half * NQH;
+    const int kl = quarter * 32 + lane;      // TMEM lane: key of S^T, dh row of O^T
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const size_t part_floats = (size_t)NQ * DH + 2 * NQ;
-    float l[NQ];
+    const float scale = p.qk_scale;
+    float l[NQH], mrun[NQH];
     int seg = -1;
     int n_draft = 0, n_side = 0;
     int pv_waited = -1;  // index of the last PV this thread waited for
@@ -289,8 +380,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (first) {
         ++seg;
         seg_t0 = t;
-        // segment metadata: running max reset, verify tables of sequence b
-        if (st < NQ) m_run[st] = -INFINITY;
+        // segment metadata: verify tables of sequence b
         if (VERIFY) {
           const int r0 = b * p.rows;
           if (st < NQ) {
@@ -322,7 +412,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
         }
 #pragma unroll
-        for (int c = 0; c < NQ; ++c) l[c] = 0.f;
+        for (int c = 0; c < NQH; ++c) {
+          l[c] = 0.f;
+          mrun[c] = -INFINITY;
+        }
         tc::named_bar_sync(1, kSmx);
         if (VERIFY) {
           n_draft = *n_draft_s;
@@ -330,29 +423,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       }
 
-      // ---- scores of this tile (thread = key kl)
+      // ---- raw scores of this tile: row kl of S^T, this thread's columns
       const int sb = i & 1;
       // after a timeout every later wait returns at once: keep going so that all
       // softmax threads still meet at the same named barriers
       tc::mbar_wait(&s_full[sb], (uint32_t)(i >> 1) & 1u, abort_flag, p.status);
       tc::tc_fence_after();
-      float s[NQ];
-      tmem_ld_row<NQ>(tmem + lane_off + sb * NQ, s);
+      float s[NQH];
+      tmem_ld_row<NQH>(tmem + lane_off + sb * NQ + c0, s);
       tc::tmem_wait_ld();
       tc::tc_fence_before();
-      tc::mbar_arrive(&s_empty[sb]);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&s_empty[sb]);
 
       const bool side_tile = VERIFY && t >= p.n_cache_tiles;
       const int key = (side_tile ? t - p.n_cache_tiles : t) * kKT + kl;
       const bool valid = key < (side_tile ? n_side : p.N);
+      if (!valid) {
 #pragma unroll
-      for (int c = 0; c < NQ; ++c) s[c] = valid ? s[c] * p.qk_scale : -INFINITY;
-      if (VERIFY && valid) {
+        for (int c = 0; c < NQH; ++c) s[c] = -INFINITY;
+      } else if (VERIFY) {
         if (side_tile) {
           const int srank = side_rank[key];
 #pragma unroll
-          for (int c = 0; c < NQ; ++c) {
-            const int cm = col_meta[c];
+          for (int c = 0; c < NQH; ++c) {
+            const int cm = col_meta[c0 + c];
             if (!visible_side(cm & 3, cm >> 2, srank, p.causal)) s[c] = -INFINITY;
           }
         } else {
@@ -361,60 +456,71 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (draft_pos[d] == key) kdr = draft_rank[d];
           if (kdr >= 0) {
 #pragma unroll
-            for (int c = 0; c < NQ; ++c) {
-              const int cm = col_meta[c];
+            for (int c = 0; c < NQH; ++c) {
+              const int cm = col_meta[c0 + c];
               if (!visible_cache(cm & 3, cm >> 2, kdr, p.causal)) s[c] = -INFINITY;
             }
           }
         }
       }
 
-      // ---- running max: raised only when a column's tile max exceeds it by 2^8
+      // ---- running max: raised only when a score exceeds it by more than 2^8
+      // (with m = -inf any finite score does; masked scores, -inf, never do)
       bool need = false;
 #pragma unroll
-      for (int c = 0; c < NQ; ++c) need |= warp_max(s[c]) > m_run[c] + kThresh;
+      for (int c = 0; c < NQH; ++c) need |= fmaf(s[c], scale, -mrun[c]) > kThresh;
       const bool any = bar_any(2, kSmx, need);
       if (any) {
 #pragma unroll
-        for (int c = 0; c < NQ; ++c) {
+        for (int c = 0; c < NQH; ++c) {
           const float wm = warp_max(s[c]);
-          if (lane == (c & 31)) wred[quarter * NQ + c] = wm;
+          if (lane == (c & 31)) wred[quarter * NQ + c0 + c] = wm * scale;
         }
         tc::named_bar_sync(1, kSmx);
         if (st < NQ) {
           const float mo = m_run[st];
           const float tm = fmaxf(fmaxf(wred[st], wred[NQ + st]), fmaxf(wred[2 * NQ + st], wred[3 * NQ + st]));
-          const float mn = (tm > mo + kThresh) ? tm : mo;
-          alpha[st] = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+          const bool first_col = first || !(mo > -INFINITY);
+          const float mcur = first_col ? -INFINITY : mo;
+          const float mn = (tm > mcur + kThresh) ? tm : mcur;
+          alpha[st] = (mcur == -INFINITY) ? 0.f : exp2f(mcur - mn);
           m_run[st] = mn;
         }
         tc::named_bar_sync(1, kSmx);
 #pragma unroll
-        for (int c = 0; c < NQ; ++c) l[c] *= alpha[c];
+        for (int c = 0; c < NQH; ++c) {
+          mrun[c] = m_run[c0 + c];
+          l[c] *= alpha[c0 + c];
+        }
       }
 
-      // ---- the previous PV must be complete: P buffer free, O stable
-      if (i > 0 && pv_waited < i - 1) {
-        tc::mbar_wait(pv_done, (uint32_t)(i - 1) & 1u, abort_flag, p.status);
+      // ---- P buffer i&1 is free once PV(i-2) is done; rescaling O needs PV(i-1)
+      if (i >= 2 && pv_waited < i - 2) {
+        tc::mbar_wait(&pv_done[i & 1], (uint32_t)((i - 2) >> 1) & 1u, abort_flag, p.status);
+        pv_waited = i - 2;
+      }
+      if (any && !first && i >= 1 && pv_waited < i - 1) {
+        tc::mbar_wait(&pv_done[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u, abort_flag, p.status);
         pv_waited = i - 1;
       }
       tc::tc_fence_after();
       if (any && !first) {
-        // rescale the O^T accumulator, column c by alpha[c]
+        // rescale this thread's columns of the O^T accumulator (row kl)
         float o[16];
 #pragma unroll
-        for (int c0 = 0; c0 < NQ; c0 += 16) {
-          tc::tmem_ld16(tmem_o + lane_off + c0, o);
+        for (int cc = 0; cc < NQH; cc += 16) {
+          tc::tmem_ld16(tmem_o + lane_off + c0 + cc, o);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 16; ++c) o[c] *= alpha[c0 + c];
-          tc::tmem_st16(tmem_o + lane_off + c0, o);
+          for (int c = 0; c < 16; ++c) o[c] *= alpha[c0 + cc + c];
+          tc::tmem_st16(tmem_o + lane_off + c0 + cc, o);
         }
         tc::tmem_wait_st();
       }
       // a side tile's key rows past the used slots may hold anything: zero them
-      if (side_tile && !valid) {
-        uint8_t* vrow = smem + (i % NS) * L::kStageBytes + L::kTileBytes + kl * 128;
+      if (side_tile && !valid && half == 0) {
+        tc::mbar_wait(&v_full[i % NV], (uint32_t)(i / NV) & 1u, abort_flag, p.status);
+        uint8_t* vrow = v_ring + (i % NV) * L::kTileBytes + kl * 128;
 #pragma unroll
         for (int x = 0; x < L::kBoxes; ++x)
 #pragma unroll
@@ -422,59 +528,63 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             *reinterpret_cast<uint4*>(vrow + x * 16384 + q * 16) = make_uint4(0u, 0u, 0u, 0u);
       }
 
-      // ---- P = exp2(s - m), row kl of the MN-major swizzled P^T tile
+      // ---- P = 2^(s*scale - m) into row kl of the MN-major swizzled P^T tile
       {
-        uint32_t pk[NQ / 2];
+        uint32_t pk[NQH / 2];
 #pragma unroll
-        for (int c = 0; c < NQ; c += 2) {
-          const float m0 = m_run[c], m1 = m_run[c + 1];
-          const float p0 = (m0 == -INFINITY) ? 0.f : exp2f(s[c] - m0);
-          const float p1 = (m1 == -INFINITY) ? 0.f : exp2f(s[c + 1] - m1);
+        for (int c = 0; c < NQH; c += 2) {
+          // fmaxf turns the NaN of (-inf) - (-inf) into -inf, i.e. p = 0
+          const float p0 = ex2_approx(fmaxf(fmaf(s[c], scale, -mrun[c]), -INFINITY));
+          const float p1 = ex2_approx(fmaxf(fmaf(s[c + 1], scale, -mrun[c + 1]), -INFINITY));
           l[c] += p0;
           l[c + 1] += p1;
           pk[c / 2] = pack_bf16x2(p0, p1);
         }
-        uint8_t* prow = p_buf + kl * L::kPRow;
         constexpr uint32_t mask = L::kPRow / 16 - 1;  // swizzle span: row bytes
 #pragma unroll
-        for (int ch = 0; ch < NQ / 8; ++ch) {
-          const uint32_t off = (uint32_t)(kl * L::kPRow + ch * 16);
+        for (int ch = 0; ch < NQH / 8; ++ch) {
+          const uint32_t off = (uint32_t)(kl * L::kPRow + (c0 * 2) + ch * 16);
           const uint32_t sw = off ^ (((off >> 7) & mask) << 4);
-          *reinterpret_cast<uint4*>(p_buf + sw) =
+          *reinterpret_cast<uint4*>(p_buf + (i & 1) * L::kPBufBytes + sw) =
               make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
         }
-        (void)prow;
       }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
-      tc::mbar_arrive(p_full);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&p_full[i & 1]);
 
       if (last) {
         // ---- segment done: O^T complete after this tile's PV
-        tc::mbar_wait(pv_done, (uint32_t)i & 1u, abort_flag, p.status);
+        tc::mbar_wait(&pv_done[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag, p.status);
         pv_waited = i;
         tc::tc_fence_after();
-        // total l per column: butterfly within each warp, then across warps
+        // total l per column: butterfly within each warp, then across quarters
 #pragma unroll
-        for (int c = 0; c < NQ; ++c) {
+        for (int c = 0; c < NQH; ++c) {
           float v = l[c];
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          if (lane == (c & 31)) wred[quarter * NQ + c] = v;
+          if (lane == (c & 31)) wred[quarter * NQ + c0 + c] = v;
+          // the next segment starts afresh: end the live ranges here
+          l[c] = 0.f;
+          mrun[c] = -INFINITY;
         }
+        if (st < NQ) alpha[st] = m_run[st];  // keep m while wred is reused below
         tc::named_bar_sync(1, kSmx);
-        float o[NQ];
-        tmem_ld_row<NQ>(tmem_o + lane_off, o);
+        float o[NQH];
+        tmem_ld_row<NQH>(tmem_o + lane_off + c0, o);
         tc::tmem_wait_ld();
         const bool whole = (seg_t0 == 0) && (t == tpi - 1);
         const int h = bh % p.H;
         if (whole) {
           if (kl < DH) {
 #pragma unroll
-            for (int c = 0; c < NQ; ++c) {
-              const int r = qc * NQ + c;
+            for (int c = 0; c < NQH; ++c) {
+              const int r = qc * NQ + c0 + c;
+              const int cq = c0 + c;
               if (r < p.rows) {
-                const float lt = wred[c] + wred[NQ + c] + wred[2 * NQ + c] + wred[3 * NQ + c];
+                const float lt = wred[cq] + wred[NQ + cq] + wred[2 * NQ + cq] + wred[3 * NQ + cq];
                 p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + kl] = __float2bfloat16_rn(o[c] / lt);
               }
             }
@@ -485,10 +595,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           float* part = p.partials + ((size_t)cta * 2 + slot) * part_floats;
           if (kl < DH) {
 #pragma unroll
-            for (int c = 0; c < NQ; ++c) part[(size_t)c * DH + kl] = o[c];
+            for (int c = 0; c < NQH; ++c) part[(size_t)(c0 + c) * DH + kl] = o[c];
           }
           if (st < NQ) {
-            part[(size_t)NQ * DH + st] = m_run[st];
+            part[(size_t)NQ * DH + st] = alpha[st];
             part[(size_t)NQ * DH + NQ + st] = wred[st] + wred[NQ + st] + wred[2 * NQ + st] + wred[3 * NQ + st];
           }
           __threadfence();
@@ -505,8 +615,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           if (*last_flag) {
             __threadfence();
             // merge the contributors' (O, m, l) in CTA order, 16 at a time:
-            // weights 2^(m - M) per column first, then every column's loads
-            // of one contributor in flight together
+            // weights 2^(m - M) per column first, then all of this thread's
+            // column loads of one contributor in flight together
             float* wts = reinterpret_cast<float*>(draft_pos);  // [16][NQ], free here
             float M = -INFINITY;
             if (st < NQ) {
@@ -516,9 +626,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               }
             }
             float lt = 0.f;
-            float acc[NQ];
+            float acc[NQH];
 #pragma unroll
-            for (int c = 0; c < NQ; ++c) acc[c] = 0.f;
+            for (int c = 0; c < NQH; ++c) acc[c] = 0.f;
             for (int g0 = c_first; g0 <= c_last; g0 += 16) {
               const int g1 = min(c_last + 1, g0 + 16);
               if (st < NQ) {
@@ -536,11 +646,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int cb = g0; cb < g1; ++cb) {
                   const int sl = (item == (int)(unit_lo(p.total_units, G, cb) / tpi)) ? 0 : 1;
                   const float* pc = p.partials + ((size_t)cb * 2 + sl) * part_floats + kl;
-                  float ov[NQ];
+                  float ov[NQH];
 #pragma unroll
-                  for (int c = 0; c < NQ; ++c) ov[c] = __ldcg(pc + (size_t)c * DH);
+                  for (int c = 0; c < NQH; ++c) ov[c] = __ldcg(pc + (size_t)(c0 + c) * DH);
 #pragma unroll
-                  for (int c = 0; c < NQ; ++c) acc[c] += wts[(cb - g0) * NQ + c] * ov[c];
+                  for (int c = 0; c < NQH; ++c) acc[c] += wts[(cb - g0) * NQ + c0 + c] * ov[c];
                 }
               }
               tc::named_bar_sync(1, kSmx);
@@ -549,10 +659,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tc::named_bar_sync(1, kSmx);
             if (kl < DH) {
 #pragma unroll
-              for (int c = 0; c < NQ; ++c) {
-                const int r = qc * NQ + c;
+              for (int c = 0; c < NQH; ++c) {
+                const int r = qc * NQ + c0 + c;
                 if (r < p.rows)
-                  p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + kl] = __float2bfloat16_rn(acc[c] / alpha[c]);
+                  p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + kl] = __float2bfloat16_rn(acc[c] / alpha[c0 + c]);
               }
             }
           }
@@ -573,7 +683,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 }
 
 struct AttnPlan {
-  int NQ, n_qc, nct, nst, tpi, nstage, grid;
+  int NQ, n_qc, nct, nst, tpi, nk, nv, grid;
   long long items, total_units;
   size_t smem_bytes, partial_bytes, counter_bytes;
 };
@@ -591,14 +701,17 @@ AttnPlan plan(int B, int N, int H, int dh, int rows, int S_max, int verify, int 
   q.total_units = q.items * q.tpi;
   q.grid = (int)(q.total_units < num_sms ? q.total_units : num_sms);
   const size_t boxes = dh / 64;
-  const size_t stage = 2 * boxes * 16384;
+  const size_t tile = boxes * 16384;
   const size_t qbytes = boxes * q.NQ * 128;
-  const size_t pbytes = ((size_t)kKT * q.NQ * 2 + 1023) / 1024 * 1024;
+  const size_t pbytes = 2 * (((size_t)kKT * q.NQ * 2 + 1023) / 1024 * 1024);
   const size_t fixed = 1024 + 2 * qbytes + pbytes + 4096 + 3 * kMaxRows * 4;
-  int ns = (int)((kSmemBudget - fixed) / stage);
-  if (ns > 8) ns = 8;
-  q.nstage = ns;
-  q.smem_bytes = fixed + (size_t)ns * stage;
+  // K and V tiles share what shared memory is left; K gets the odd one
+  int tiles = (int)((kSmemBudget - fixed) / tile);
+  if (tiles > 16) tiles = 16;
+  q.nv = tiles / 2;
+  q.nk = tiles - q.nv;
+  if (q.nk > 8) q.nk = 8;
+  q.smem_bytes = fixed + (size_t)(q.nk + q.nv) * tile;
   q.partial_bytes = align_up((size_t)q.grid * 2 * ((size_t)q.NQ * dh + 2 * q.NQ) * sizeof(float), 256);
   q.counter_bytes = align_up((size_t)q.items * sizeof(unsigned), 256);
   return q;
@@ -611,7 +724,7 @@ cudaError_t launch_t(const AttnArgs& a, const AttnPlan& q, AttnTcParams prm, con
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)q.smem_bytes);
   if (e != cudaSuccess) return e;
-  kern<<<q.grid, kThreads, q.smem_bytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], prm);
+  kern<<<q.grid, Threads<NQ>::kAll, q.smem_bytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], prm);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -629,7 +742,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   if (a.B * a.rows_per_seq == 0) return cudaSuccess;
   if (a.verify && a.rows_per_seq > kMaxRows) return cudaErrorInvalidValue;
   const AttnPlan q = plan(a.B, a.N, a.H, a.dh, a.rows_per_seq, a.S_max, a.verify, device_sm_count());
-  if (q.nstage < 2) return cudaErrorInvalidValue;
+  if (q.nk < 2 || q.nv < 2) return cudaErrorInvalidValue;
   if (q.partial_bytes + q.counter_bytes > a.ws_bytes) return cudaErrorInvalidValue;
   const int dh = a.dh, E = a.H * a.dh;
   CUtensorMap maps[5];
@@ -660,7 +773,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   prm.B = a.B; prm.N = a.N; prm.H = a.H; prm.rows = a.rows_per_seq; prm.S_max = a.S_max;
   prm.causal = a.causal_cross;
   prm.n_qc = q.n_qc; prm.n_cache_tiles = q.nct; prm.n_side_tiles = q.nst; prm.tpi = q.tpi;
-  prm.nstage = q.nstage; prm.total_units = q.total_units;
+  prm.nk = q.nk; prm.nv = q.nv; prm.total_units = q.total_units;
   prm.qk_scale = kLog2e / sqrtf((float)dh);
   prm.pos = a.pos; prm.view = a.view; prm.rank = a.rank;
   prm.out = static_cast<__nv_bfloat16*>(a.out);

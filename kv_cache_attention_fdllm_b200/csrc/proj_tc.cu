@@ -155,7 +155,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&acc_full[b], 1);
-      tc::mbar_init(&acc_empty[b], kEpiThreads);
+      tc::mbar_init(&acc_empty[b], kEpiThreads / 32);  // one arrival per epilogue warp
     }
     *abort_flag = 0;
     tc::fence_mbar_init();
@@ -316,7 +316,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             if (cc + n < BN) dst[(size_t)(cc + n) * kBM + f_loc] = v[n];
         }
         tc::tc_fence_before();
-        tc::mbar_arrive(&acc_empty[buf]);
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&acc_empty[buf]);
         __threadfence();
         const long long tu0 = (long long)tile * p.nks;
         c_first = owner_of(tu0, p.total_units, G);
@@ -427,7 +428,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       }
       if (whole) {
         tc::tc_fence_before();
-        tc::mbar_arrive(&acc_empty[buf]);
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&acc_empty[buf]);
       }
     }
   }
