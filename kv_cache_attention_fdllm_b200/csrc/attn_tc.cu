@@ -56,13 +56,39 @@ struct AttnTcParams {
 __device__ __forceinline__ long long unit_lo(long long total, int G, int c) {
   return total * c / G;
 }
+// The CTA whose unit range holds unit u: the largest c with unit_lo(c) <= u,
+// i.e. total * c < (u + 1) * G.  A double-precision estimate is corrected with
+// exact 64-bit products (64-bit integer division is a long software routine).
 __device__ __forceinline__ int owner_of(long long u, long long total, int G) {
-  int c = (int)(((u + 1) * G - 1) / total);
-  if (c >= G) c = G - 1;
-  while (c > 0 && unit_lo(total, G, c) > u) --c;
-  while (c + 1 < G && unit_lo(total, G, c + 1) <= u) ++c;
+  const long long lim = (u + 1) * (long long)G;
+  int c = (int)((double)(lim - 1) / (double)total);
+  c = c < 0 ? 0 : (c >= G ? G - 1 : c);
+  while (c + 1 < G && total * (c + 1) < lim) ++c;
+  while (c > 0 && total * c >= lim) --c;
   return c;
 }
+
+// (item, tile within the item, query chunk, sequence*head) of a unit, advanced
+// one unit at a time without division.
+struct UnitCursor {
+  int item, t, qc, bh;
+  __device__ __forceinline__ void init(long long u, int tpi, int n_qc) {
+    item = (int)(u / tpi);
+    t = (int)(u - (long long)item * tpi);
+    bh = item / n_qc;
+    qc = item - bh * n_qc;
+  }
+  __device__ __forceinline__ void next(int tpi, int n_qc) {
+    if (++t == tpi) {
+      t = 0;
+      ++item;
+      if (++qc == n_qc) {
+        qc = 0;
+        ++bh;
+      }
+    }
+  }
+};
 
 __device__ __forceinline__ float warp_max(float v) {
   float r;
@@ -232,13 +258,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const uint64_t pol_kv = tc::policy_evict_first();
       const uint64_t pol_q = tc::policy_evict_last();
       int ik = 0, iv = 0, seg = -1;
+      UnitCursor ck, cv;
+      ck.init(u0, tpi, p.n_qc);
+      cv = ck;
       IdleClock clk;
       while (iv < T) {
         bool progressed = false;
         if (ik < T) {
-          const long long u = u0 + ik;
-          const int item = (int)(u / tpi), t = (int)(u % tpi);
-          const int qc = item % p.n_qc, bh = item / p.n_qc;
+          const int t = ck.t, qc = ck.qc, bh = ck.bh;
           const bool first = (ik == 0 || t == 0);
           const int qb = (seg + 1) & 1;
           const int ks = ik % NK;
@@ -260,15 +287,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int x = 0; x < L::kBoxes; ++x)
               tc::tma_load_3d(kd + x * 16384, side ? &tm_ks : &tm_k, &k_full[ks], x * 64, key0, bh, pol_kv);
             ++ik;
+            ck.next(tpi, p.n_qc);
             progressed = true;
           }
         }
         if (iv < ik) {
           const int vs = iv % NV;
           if (tc::mbar_test(&v_empty[vs], ((uint32_t)(iv / NV) & 1u) ^ 1u)) {
-            const long long u = u0 + iv;
-            const int item = (int)(u / tpi), t = (int)(u % tpi);
-            const int bh = item / p.n_qc;
+            const int t = cv.t, bh = cv.bh;
             const bool side = VERIFY && t >= p.n_cache_tiles;
             const int key0 = (side ? t - p.n_cache_tiles : t) * kKT;
             uint8_t* vd = v_ring + vs * L::kTileBytes;
@@ -277,6 +303,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int x = 0; x < L::kBoxes; ++x)
               tc::tma_load_3d(vd + x * 16384, side ? &tm_vs : &tm_v, &v_full[vs], x * 64, key0, bh, pol_kv);
             ++iv;
+            cv.next(tpi, p.n_qc);
             progressed = true;
           }
         }
@@ -294,12 +321,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       constexpr uint32_t p_swz = NQ == 64 ? 2u : (NQ == 32 ? 4u : 6u);
       const uint32_t p_addr = tc::smem_u32(p_buf);
       int iq = 0, ip = 0, seg = -1;
+      UnitCursor cq, cpv;
+      cq.init(u0, tpi, p.n_qc);
+      cpv = cq;
       IdleClock clk;
       while (ip < T) {
         bool progressed = false;
         if (iq < T) {
-          const long long u = u0 + iq;
-          const int t = (int)(u % tpi);
+          const int t = cq.t;
           const bool first = (iq == 0 || t == 0);
           const bool last = (iq == T - 1 || t == tpi - 1);
           const int qb = first ? ((seg + 1) & 1) : (seg & 1);
@@ -323,6 +352,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tc::mma_commit(&k_empty[ks]);
             if (last) tc::mma_commit(&q_empty[qb]);
             ++iq;
+            cq.next(tpi, p.n_qc);
             progressed = true;
           }
         }
@@ -330,8 +360,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const int vs = ip % NV;
           if (tc::mbar_test(&p_full[ip & 1], (uint32_t)(ip >> 1) & 1u) &&
               tc::mbar_test(&v_full[vs], (uint32_t)(ip / NV) & 1u)) {
-            const long long u = u0 + ip;
-            const bool first = (ip == 0 || (u % tpi) == 0);
+            const bool first = (ip == 0 || cpv.t == 0);
             tc::tc_fence_after();
             const uint32_t v_addr = tc::smem_u32(v_ring + vs * L::kTileBytes);
             const uint32_t pb_addr = p_addr + (ip & 1) * L::kPBufBytes;
@@ -344,6 +373,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tc::mma_commit(&pv_done[ip & 1]);
             tc::mma_commit(&v_empty[vs]);
             ++ip;
+            cpv.next(tpi, p.n_qc);
             progressed = true;
           }
         }
@@ -370,12 +400,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     int n_draft = 0, n_side = 0;
     int pv_waited = -1;  // index of the last PV this thread waited for
     int seg_t0 = 0;      // tile index at which the current segment started
-    for (int i = 0; i < T; ++i) {
-      const long long u = u0 + i;
-      const int item = (int)(u / tpi), t = (int)(u % tpi);
+    UnitCursor cs;
+    cs.init(u0, tpi, p.n_qc);
+    const int item0 = cs.item;
+    for (int i = 0; i < T; ++i, cs.next(tpi, p.n_qc)) {
+      const int item = cs.item, t = cs.t, qc = cs.qc, bh = cs.bh;
       const bool first = (i == 0 || t == 0);
       const bool last = (i == T - 1 || t == tpi - 1);
-      const int qc = item % p.n_qc, bh = item / p.n_qc;
       const int b = bh / p.H;
       if (first) {
         ++seg;
@@ -590,12 +621,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
           }
         } else {
-          // partial item: (O, m, l) to this CTA's slot; the last contributor merges
-          const int slot = (item == (int)(u0 / tpi)) ? 0 : 1;
+          // partial item: (O, m, l) to this CTA's slot; the last contributor merges.
+          // Slot: O as [dh row][NQ columns] (a thread's 16 columns are 64
+          // contiguous bytes), then m[NQ], then l[NQ].
+          const int slot = (item == item0) ? 0 : 1;
           float* part = p.partials + ((size_t)cta * 2 + slot) * part_floats;
           if (kl < DH) {
+            float4* dst = reinterpret_cast<float4*>(part + (size_t)kl * NQ + c0);
 #pragma unroll
-            for (int c = 0; c < NQH; ++c) part[(size_t)(c0 + c) * DH + kl] = o[c];
+            for (int v = 0; v < NQH / 4; ++v)
+              dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
           }
           if (st < NQ) {
             part[(size_t)NQ * DH + st] = alpha[st];
@@ -614,55 +649,101 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tc::named_bar_sync(1, kSmx);
           if (*last_flag) {
             __threadfence();
-            // merge the contributors' (O, m, l) in CTA order, 16 at a time:
-            // weights 2^(m - M) per column first, then all of this thread's
-            // column loads of one contributor in flight together
-            float* wts = reinterpret_cast<float*>(draft_pos);  // [16][NQ], free here
-            float M = -INFINITY;
+            // Merge the contributors in CTA order.  The loads of a batch are
+            // all issued before any is used, so the merge costs a few L2 round
+            // trips, not a few per contributor.
+            //   (1) per column: M = max m_j, L = sum 2^(m_j - M) l_j (8 at a time)
+            //   (2) O = sum (2^(m_j - M) / L) O_j, weights staged in shared memory
+            const int n_c = c_last - c_first + 1;
+            // slot 0 when the item is the contributor's first, i.e. its range
+            // starts inside the item: unit_lo(cb) >= iu0 <=> total * cb >= iu0 * G
+            const long long lim0 = iu0 * (long long)G;
+            auto part_of = [&](int cb) -> const float* {
+              const int sl = (p.total_units * cb >= lim0) ? 0 : 1;
+              return p.partials + ((size_t)cb * 2 + sl) * part_floats;
+            };
+            float* wts = reinterpret_cast<float*>(draft_pos);  // [8][NQ], free here
+            float M = -INFINITY, Lsum = 0.f;
+            float mv[8];
             if (st < NQ) {
-              for (int cb = c_first; cb <= c_last; ++cb) {
-                const int sl = (item == (int)(unit_lo(p.total_units, G, cb) / tpi)) ? 0 : 1;
-                M = fmaxf(M, __ldcg(p.partials + ((size_t)cb * 2 + sl) * part_floats + (size_t)NQ * DH + st));
+              for (int g0 = 0; g0 < n_c; g0 += 8) {
+                float lv[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  mv[j] = -INFINITY;
+                  lv[j] = 0.f;
+                  if (g0 + j < n_c) {
+                    const float* pc = part_of(c_first + g0 + j);
+                    mv[j] = __ldcg(pc + (size_t)NQ * DH + st);
+                    lv[j] = __ldcg(pc + (size_t)NQ * DH + NQ + st);
+                  }
+                }
+                float mc = M;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) mc = fmaxf(mc, mv[j]);
+                if (mc > -INFINITY) {
+                  Lsum *= (M == -INFINITY) ? 0.f : exp2f(M - mc);
+#pragma unroll
+                  for (int j = 0; j < 8; ++j) Lsum += (mv[j] == -INFINITY) ? 0.f : exp2f(mv[j] - mc) * lv[j];
+                  M = mc;
+                }
               }
             }
-            float lt = 0.f;
+            constexpr int kJ = NQ == 64 ? 2 : 4;  // contributors per batch of O loads
             float acc[NQH];
 #pragma unroll
             for (int c = 0; c < NQH; ++c) acc[c] = 0.f;
-            for (int g0 = c_first; g0 <= c_last; g0 += 16) {
-              const int g1 = min(c_last + 1, g0 + 16);
+            for (int g0 = 0; g0 < n_c; g0 += 8) {
               if (st < NQ) {
-                for (int cb = g0; cb < g1; ++cb) {
-                  const int sl = (item == (int)(unit_lo(p.total_units, G, cb) / tpi)) ? 0 : 1;
-                  const float* pc = p.partials + ((size_t)cb * 2 + sl) * part_floats;
-                  const float mc = __ldcg(pc + (size_t)NQ * DH + st);
-                  const float w = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
-                  lt += w * __ldcg(pc + (size_t)NQ * DH + NQ + st);
-                  wts[(cb - g0) * NQ + st] = w;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  float m = mv[j];
+                  if (n_c > 8) m = (g0 + j < n_c) ? __ldcg(part_of(c_first + g0 + j) + (size_t)NQ * DH + st) : -INFINITY;
+                  wts[j * NQ + st] = (m == -INFINITY || !(Lsum > 0.f)) ? 0.f : exp2f(m - M) / Lsum;
                 }
               }
               tc::named_bar_sync(1, kSmx);
               if (kl < DH) {
-                for (int cb = g0; cb < g1; ++cb) {
-                  const int sl = (item == (int)(unit_lo(p.total_units, G, cb) / tpi)) ? 0 : 1;
-                  const float* pc = p.partials + ((size_t)cb * 2 + sl) * part_floats + kl;
-                  float ov[NQH];
+                const int nj = min(8, n_c - g0);
+                for (int j0 = 0; j0 < nj; j0 += kJ) {
+                  float4 ov[kJ][NQH / 4];
 #pragma unroll
-                  for (int c = 0; c < NQH; ++c) ov[c] = __ldcg(pc + (size_t)(c0 + c) * DH);
+                  for (int j = 0; j < kJ; ++j) {
+                    if (j0 + j < nj) {
+                      const float4* src = reinterpret_cast<const float4*>(part_of(c_first + g0 + j0 + j) + (size_t)kl * NQ + c0);
 #pragma unroll
-                  for (int c = 0; c < NQH; ++c) acc[c] += wts[(cb - g0) * NQ + c0 + c] * ov[c];
+                      for (int v = 0; v < NQH / 4; ++v) ov[j][v] = __ldcg(src + v);
+                    } else {
+#pragma unroll
+                      for (int v = 0; v < NQH / 4; ++v) ov[j][v] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                  }
+#pragma unroll
+                  for (int j = 0; j < kJ; ++j) {
+                    const float* wj = wts + (j0 + j) * NQ + c0;
+#pragma unroll
+                    for (int v = 0; v < NQH / 4; ++v) {
+                      // weights past nj are stale but multiply zeros
+                      const float w0 = (j0 + j < nj) ? wj[4 * v] : 0.f;
+                      const float w1 = (j0 + j < nj) ? wj[4 * v + 1] : 0.f;
+                      const float w2 = (j0 + j < nj) ? wj[4 * v + 2] : 0.f;
+                      const float w3 = (j0 + j < nj) ? wj[4 * v + 3] : 0.f;
+                      acc[4 * v] = fmaf(w0, ov[j][v].x, acc[4 * v]);
+                      acc[4 * v + 1] = fmaf(w1, ov[j][v].y, acc[4 * v + 1]);
+                      acc[4 * v + 2] = fmaf(w2, ov[j][v].z, acc[4 * v + 2]);
+                      acc[4 * v + 3] = fmaf(w3, ov[j][v].w, acc[4 * v + 3]);
+                    }
+                  }
                 }
               }
               tc::named_bar_sync(1, kSmx);
             }
-            if (st < NQ) alpha[st] = lt;
-            tc::named_bar_sync(1, kSmx);
             if (kl < DH) {
 #pragma unroll
               for (int c = 0; c < NQH; ++c) {
                 const int r = qc * NQ + c0 + c;
                 if (r < p.rows)
-                  p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + kl] = __float2bfloat16_rn(acc[c] / alpha[c0 + c]);
+                  p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + kl] = __float2bfloat16_rn(acc[c]);
               }
             }
           }

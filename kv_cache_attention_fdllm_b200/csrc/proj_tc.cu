@@ -77,12 +77,15 @@ struct ProjTcParams {
 __device__ __forceinline__ long long unit_lo(long long total, int G, int c) {
   return total * c / G;
 }
-// The CTA whose unit range holds unit u.
+// The CTA whose unit range holds unit u: the largest c with unit_lo(c) <= u,
+// i.e. total * c < (u + 1) * G.  A double-precision estimate is corrected with
+// exact 64-bit products (64-bit integer division is a long software routine).
 __device__ __forceinline__ int owner_of(long long u, long long total, int G) {
-  int c = (int)(((u + 1) * G - 1) / total);
-  if (c >= G) c = G - 1;
-  while (c > 0 && unit_lo(total, G, c) > u) --c;
-  while (c + 1 < G && unit_lo(total, G, c + 1) <= u) ++c;
+  const long long lim = (u + 1) * (long long)G;
+  int c = (int)((double)(lim - 1) / (double)total);
+  c = c < 0 ? 0 : (c >= G ? G - 1 : c);
+  while (c + 1 < G && total * (c + 1) < lim) ++c;
+  while (c > 0 && total * c >= lim) --c;
   return c;
 }
 
@@ -144,6 +147,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   const int G = gridDim.x, c = blockIdx.x;
   const long long u_begin = unit_lo(p.total_units, G, c);
   const long long u_end = unit_lo(p.total_units, G, c + 1);
+  // (tile, k-step) of the first unit; later units are reached by stepping
+  const int tile_begin = (int)(u_begin / p.nks);
+  const int ks_begin = (int)(u_begin - (long long)tile_begin * p.nks);
 
   uint32_t ncols = 32;
   while ((int)ncols < 2 * BN) ncols <<= 1;
@@ -177,9 +183,12 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       // W does not depend on the prep kernel: fill the first stages before
       // waiting for it, then add their X boxes.
       const int pre = (int)(n_units < p.nstage ? n_units : p.nstage);
+      int tile = tile_begin, ks = ks_begin;
       for (int i = 0; i < pre; ++i) {
-        const long long u = u_begin + i;
-        const int tile = (int)(u / p.nks), ks = (int)(u % p.nks);
+        if (i > 0 && ++ks == p.nks) {
+          ks = 0;
+          ++tile;
+        }
         const int sb0 = ks * p.subs, nsub = min(p.subs, p.nsub_total - sb0);
         uint8_t* a_s = smem + i * stage_bytes;
         tc::mbar_arrive_expect_tx(&full[i], (uint32_t)nsub * (kASubBytes + bsub_bytes));
@@ -188,21 +197,27 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                           (tile / p.n_tt) * kBM, pol_w);
       }
       grid_dep_wait();
+      tile = tile_begin;
+      ks = ks_begin;
       for (int i = 0; i < pre; ++i) {
-        const long long u = u_begin + i;
-        const int tile = (int)(u / p.nks), ks = (int)(u % p.nks);
+        if (i > 0 && ++ks == p.nks) {
+          ks = 0;
+          ++tile;
+        }
         const int sb0 = ks * p.subs, nsub = min(p.subs, p.nsub_total - sb0);
         uint8_t* b_s = smem + i * stage_bytes + p.subs * kASubBytes;
         for (int q = 0; q < nsub; ++q)
           tc::tma_load_2d(b_s + q * bsub_bytes, &tm_x, &full[i], (sb0 + q) * kSub,
                           (tile % p.n_tt) * BN, pol_x);
       }
-      for (long long u = u_begin + pre; u < u_end; ++u) {
-        const int it = (int)(u - u_begin);
+      for (int it = pre; it < (int)n_units; ++it) {
+        if (++ks == p.nks) {
+          ks = 0;
+          ++tile;
+        }
         const int s = it % p.nstage;
         const uint32_t ph = (uint32_t)(it / p.nstage) & 1u;
         if (!tc::mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status)) break;
-        const int tile = (int)(u / p.nks), ks = (int)(u % p.nks);
         const int sb0 = ks * p.subs, nsub = min(p.subs, p.nsub_total - sb0);
         uint8_t* a_s = smem + s * stage_bytes;
         uint8_t* b_s = a_s + p.subs * kASubBytes;
@@ -223,7 +238,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       int it = 0, j = 0;
       bool ok = true;
       for (long long u = u_begin; u < u_end && ok; ++j) {
-        const int ks0 = (int)(u % p.nks);
+        const int ks0 = (u == u_begin) ? ks_begin : 0;  // later segments start a tile
         const int ks1 = (int)min((long long)p.nks, ks0 + (u_end - u));
         u += ks1 - ks0;
         const int buf = j & 1;
@@ -264,8 +279,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     float* my_parts = p.partials + (size_t)c * 2 * BN * kBM;
     int j = 0;
     for (long long u = u_begin; u < u_end; ++j) {
-      const int tile = (int)(u / p.nks);
-      const int ks0 = (int)(u % p.nks);
+      const int tile = tile_begin + j;  // a segment is the part of one tile
+      const int ks0 = (j == 0) ? ks_begin : 0;
       const int ks1 = (int)min((long long)p.nks, ks0 + (u_end - u));
       u += ks1 - ks0;
       const int buf = j & 1;
@@ -303,9 +318,10 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
 
       bool run = true;
       int c_first = c, c_last = c;
+      const long long tu0 = (long long)tile * p.nks;
       if (!whole) {
         // partial tile: store it, free the accumulator, and see who is last
-        const int slot = (tile == (int)(u_begin / p.nks)) ? 0 : 1;
+        const int slot = (j == 0) ? 0 : 1;
         float* dst = my_parts + (size_t)slot * BN * kBM;
         for (int cc = 0; cc < BN; cc += kChunk) {
           float v[kChunk];
@@ -319,7 +335,6 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&acc_empty[buf]);
         __threadfence();
-        const long long tu0 = (long long)tile * p.nks;
         c_first = owner_of(tu0, p.total_units, G);
         c_last = owner_of(tu0 + p.nks - 1, p.total_units, G);
         tc::named_bar_sync(1, kEpiThreads);
@@ -353,7 +368,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             const int f4 = (etid & 31) * 4;
             const int nb = etid >> 5;  // tokens nb, nb + 4, ...
             for (int cb = c_first; cb <= c_last; ++cb) {
-              const int sl = (tile == (int)(unit_lo(p.total_units, G, cb) / p.nks)) ? 0 : 1;
+              // slot 0 when the tile is cb's first: unit_lo(cb) >= tu0
+              const int sl = (p.total_units * cb >= tu0 * (long long)G) ? 0 : 1;
               const float* ps = p.partials + ((size_t)cb * 2 + sl) * BN * kBM;
 #pragma unroll
               for (int i = 0; i < 8; ++i) {

@@ -74,6 +74,14 @@ def test_ragged_shapes(F, dtype, dh, shape):
     _check_fused(F, inp)
 
 
+@pytest.mark.parametrize("shape", [(1, 4096, 128, 1, 128, 20), (1, 6000, 128, 2, 64, 40)])
+def test_item_split_over_many_ctas(F, shape):
+    """Few (sequence, head) items and a long cache: each item's key tiles are
+    spread over dozens of CTAs, so the partial merge runs in several batches."""
+    B, N, D, H, dh, nq = shape
+    _check_fused(F, W.random_fused(B, N, D, H, dh, nq=nq, seed=N + H))
+
+
 def test_edge_slots_and_single_query(F):
     N = 257
     q_idx = np.array([[0, N - 1, 128], [N - 1, 5, 0]], np.int32)
