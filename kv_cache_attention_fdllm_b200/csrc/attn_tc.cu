@@ -16,11 +16,18 @@
 // are then rescaled), so most tiles need no rescaling; P goes to shared memory
 // as bf16 in the MN-major swizzled layout the PV MMA reads.
 //
-// Persistent stream-K: one CTA per SM; units (item = (sequence, head, query
-// chunk), 128-key tile) are laid out item after item and every CTA takes an
-// equal contiguous range, so the cache stream is balanced whatever B, H, N.
-// An item split between CTAs leaves (O, m, l) partials; its last contributor
-// (atomic counter) merges them in CTA order and writes the output.
+// Two ways to spread the units (item = (sequence, head, query chunk), 128-key
+// tile) over the SMs:
+//   cluster mode (few items): one thread-block cluster of cs <= 8 CTAs per
+//     item, each CTA an equal share of its tiles.  The CTAs leave their (O, m,
+//     l) partials in their own shared memory and, after a cluster barrier,
+//     each merges a slice of the head dimension reading the others' partials
+//     through distributed shared memory.
+//   persistent stream-K (many items): one CTA per SM; units are laid out item
+//     after item and every CTA takes an equal contiguous range, so the cache
+//     stream is balanced whatever B, H, N.  An item split between CTAs leaves
+//     (O, m, l) partials in global memory; its last contributor (atomic
+//     counter) merges them in CTA order and writes the output.
 //
 //   warp 0      TMA producer: Q chunk per item, K and V tiles (128 x 64 boxes)
 //   warp 1      TMEM allocation; lane 0 issues QK (ahead by one tile) and PV
@@ -38,6 +45,7 @@ constexpr int kKT = 128;  // keys per tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kThresh = 8.f;  // lazy rescale threshold (log2 units)
 constexpr int kMaxRows = 512;   // verify rows per sequence held in shared memory
+constexpr int kL2PrefetchTiles = 4;  // cache tiles per CTA warmed in L2 before the dependency wait
 
 struct AttnTcParams {
   int B, N, H, rows, S_max, causal;
@@ -47,8 +55,11 @@ struct AttnTcParams {
   const int32_t* pos;
   const int8_t* view;
   const int32_t* rank;
+  const __nv_bfloat16* k_cache;  // [B, H, N, DH], for the L2 prefetch
+  const __nv_bfloat16* v_cache;
   __nv_bfloat16* out;
   int* status;
+  int cs;              // cluster size in cluster mode, 0 in stream-K mode
   float* partials;     // [grid][2][NQ*DH + 2*NQ]
   unsigned* item_cnt;  // [items], zero between calls
 };
@@ -209,10 +220,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
-  const long long u0 = unit_lo(p.total_units, G, cta);
-  const long long u1 = unit_lo(p.total_units, G, cta + 1);
-  const int T = (int)(u1 - u0);
   const int tpi = p.tpi;
+  const bool clustered = p.cs > 1;
+  int crank = 0;
+  long long u0, u1;
+  if (clustered) {
+    // cluster (cs, 1, 1): item blockIdx.x / cs, this CTA's share of its tiles
+    crank = (int)tc::cluster_ctarank();
+    const long long base = (long long)(cta / p.cs) * tpi;
+    u0 = base + (crank * tpi) / p.cs;
+    u1 = base + ((crank + 1) * tpi) / p.cs;
+  } else {
+    u0 = unit_lo(p.total_units, G, cta);
+    u1 = unit_lo(p.total_units, G, cta + 1);
+  }
+  const int T = (int)(u1 - u0);
 
   uint32_t ncols = 32;
   while ((int)ncols < 3 * NQ) ncols <<= 1;
@@ -240,11 +262,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc::fence_mbar_init();
   }
   if (warp == 1) tc::tmem_alloc(tmem_slot, ncols);
+  if (tid == 32 * 2) {
+    // Launched as a programmatic dependent of the projection: warm L2 with the
+    // first cache tiles of this CTA while that grid finishes (safe before the
+    // wait: L2 is where the projection's k, v writes land), then wait for it.
+    tc::prefetch_tmap(&tm_q);
+    tc::prefetch_tmap(&tm_k);
+    tc::prefetch_tmap(&tm_v);
+    UnitCursor cur;
+    cur.init(u0, tpi, p.n_qc);
+    const int npre = T < kL2PrefetchTiles ? T : kL2PrefetchTiles;
+    for (int i = 0; i < npre; ++i, cur.next(tpi, p.n_qc)) {
+      if (cur.t < p.n_cache_tiles) {
+        const int key0 = cur.t * kKT;
+        const int rows = p.N - key0 < kKT ? p.N - key0 : kKT;
+        const size_t off = ((size_t)cur.bh * p.N + key0) * DH;
+        tc::prefetch_l2(p.k_cache + off, (uint32_t)rows * DH * 2u);
+        tc::prefetch_l2(p.v_cache + off, (uint32_t)rows * DH * 2u);
+      }
+    }
+  }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tmem_o = tmem + 2 * NQ;
+  // every thread: nothing written by an earlier kernel is read before this
+  tc::griddep_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -620,6 +664,89 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               }
             }
           }
+        } else if (clustered) {
+          // ---- cluster merge.  The rings are idle (the last PV is done), so
+          // this CTA's partial goes to the start of the K ring: O^T as
+          // [dh row][NQ + 4] (the pad keeps 16-byte reads of rows at a 144-
+          // or 272-byte stride off each other's banks), then m[NQ], l[NQ].
+          constexpr int kP = NQ + 4;
+          float* cpart = reinterpret_cast<float*>(k_ring);
+          if (kl < DH) {
+            float4* dst = reinterpret_cast<float4*>(cpart + kl * kP + c0);
+#pragma unroll
+            for (int v = 0; v < NQH / 4; ++v)
+              dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          }
+          if (st < NQ) {
+            cpart[DH * kP + st] = alpha[st];
+            cpart[DH * kP + NQ + st] = wred[st] + wred[NQ + st] + wred[2 * NQ + st] + wred[3 * NQ + st];
+          }
+          tc::cluster_sync();
+          const int cs = p.cs;
+          const uint32_t cbase = tc::smem_u32(cpart);
+          // This CTA merges its slice of dh rows.  A thread takes one row and 4
+          // columns (consecutive threads: consecutive rows, so the output
+          // stores coalesce) and loads (m, l, O) of those columns from up to 4
+          // CTAs at once, merging online: one round trip per 4 CTAs.
+          const int r0 = (crank * DH) / cs, nr = ((crank + 1) * DH) / cs - r0;
+          for (int idx = st; idx < nr * (NQ / 4); idx += kSmx) {
+            const int row = r0 + idx % nr, c4 = (idx / nr) * 4;
+            float M[4], Lsum[4], acc[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              M[e] = -INFINITY;
+              Lsum[e] = 0.f;
+              acc[e] = 0.f;
+            }
+            for (int g = 0; g < cs; g += 4) {
+              float4 mv[4], lv[4], ov[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                if (g + j < cs) {
+                  const uint32_t a = tc::map_peer(cbase, (uint32_t)(g + j));
+                  mv[j] = tc::ld_peer_f32x4(a + (uint32_t)(DH * kP + c4) * 4u);
+                  lv[j] = tc::ld_peer_f32x4(a + (uint32_t)(DH * kP + NQ + c4) * 4u);
+                  ov[j] = tc::ld_peer_f32x4(a + (uint32_t)(row * kP + c4) * 4u);
+                } else {
+                  mv[j] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+                  lv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                  ov[j] = lv[j];
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                float mj[4], lj[4], oj[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  mj[j] = e == 0 ? mv[j].x : e == 1 ? mv[j].y : e == 2 ? mv[j].z : mv[j].w;
+                  lj[j] = e == 0 ? lv[j].x : e == 1 ? lv[j].y : e == 2 ? lv[j].z : lv[j].w;
+                  oj[j] = e == 0 ? ov[j].x : e == 1 ? ov[j].y : e == 2 ? ov[j].z : ov[j].w;
+                }
+                const float mn = fmaxf(fmaxf(M[e], fmaxf(mj[0], mj[1])), fmaxf(mj[2], mj[3]));
+                if (mn > -INFINITY) {
+                  const float sc = (M[e] == -INFINITY) ? 0.f : exp2f(M[e] - mn);
+                  Lsum[e] *= sc;
+                  acc[e] *= sc;
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) {
+                    const float w = (mj[j] == -INFINITY) ? 0.f : exp2f(mj[j] - mn);
+                    Lsum[e] = fmaf(w, lj[j], Lsum[e]);
+                    acc[e] = fmaf(w, oj[j], acc[e]);
+                  }
+                  M[e] = mn;
+                }
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int r = qc * NQ + c4 + e;
+              if (r < p.rows)
+                p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + row] =
+                    __float2bfloat16_rn(Lsum[e] > 0.f ? acc[e] / Lsum[e] : 0.f);
+            }
+          }
+          // no CTA leaves while another may still read its shared memory
+          tc::cluster_sync();
         } else {
           // partial item: (O, m, l) to this CTA's slot; the last contributor merges.
           // Slot: O as [dh row][NQ columns] (a thread's 16 columns are 64
@@ -754,6 +881,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   }
 
+  // the softmax warps meet the two cluster barriers of the merge; the producer
+  // and MMA warps, done with their loops, meet them here
+  if (clustered && warp < 2) {
+    tc::cluster_sync();
+    tc::cluster_sync();
+  }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -764,7 +897,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 }
 
 struct AttnPlan {
-  int NQ, n_qc, nct, nst, tpi, nk, nv, grid;
+  int NQ, n_qc, nct, nst, tpi, nk, nv, grid;  // grid: stream-K grid
+  int cs;                                      // cluster size wanted (0: stream-K)
   long long items, total_units;
   size_t smem_bytes, partial_bytes, counter_bytes;
 };
@@ -781,6 +915,14 @@ AttnPlan plan(int B, int N, int H, int dh, int rows, int S_max, int verify, int 
   q.items = (long long)B * H * q.n_qc;
   q.total_units = q.items * q.tpi;
   q.grid = (int)(q.total_units < num_sms ? q.total_units : num_sms);
+  // few items: a cluster of cs CTAs per item, merging through shared memory
+  q.cs = 0;
+  if (q.items * 2 <= num_sms) {
+    int cs = (int)(num_sms / q.items);
+    cs = cs > 8 ? 8 : cs;
+    cs = cs > q.tpi ? q.tpi : cs;
+    if (cs >= 2) q.cs = cs;
+  }
   const size_t boxes = dh / 64;
   const size_t tile = boxes * 16384;
   const size_t qbytes = boxes * q.NQ * 128;
@@ -798,6 +940,32 @@ AttnPlan plan(int B, int N, int H, int dh, int rows, int S_max, int verify, int 
   return q;
 }
 
+// How many clusters of cs CTAs of this kernel can be resident at once (cached).
+template <int NQ, int DH, bool VERIFY>
+int max_clusters(int cs, size_t smem_bytes) {
+  static int cache[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+  if (cache[cs] == 0) {
+    cudaLaunchConfig_t c = {};
+    c.gridDim = dim3(cs * 16);
+    c.blockDim = dim3(Threads<NQ>::kAll);
+    c.dynamicSmemBytes = smem_bytes;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    c.attrs = at;
+    c.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel<NQ, DH, VERIFY>, &c) != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    cache[cs] = n > 0 ? n : -1;
+  }
+  return cache[cs];
+}
+
 template <int NQ, int DH, bool VERIFY>
 cudaError_t launch_t(const AttnArgs& a, const AttnPlan& q, AttnTcParams prm, const CUtensorMap* maps,
                      cudaStream_t stream) {
@@ -805,9 +973,33 @@ cudaError_t launch_t(const AttnArgs& a, const AttnPlan& q, AttnTcParams prm, con
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)q.smem_bytes);
   if (e != cudaSuccess) return e;
-  kern<<<q.grid, Threads<NQ>::kAll, q.smem_bytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], prm);
+  // cluster mode only when every item's cluster fits in one wave
+  int cs = q.cs;
+  while (cs >= 2 && max_clusters<NQ, DH, VERIFY>(cs, q.smem_bytes) < q.items) --cs;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(Threads<NQ>::kAll);
+  cfg.dynamicSmemBytes = q.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cs >= 2) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cs;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+    cfg.gridDim = dim3((unsigned)(q.items * cs));
+    prm.cs = cs;
+  } else {
+    cfg.gridDim = dim3(q.grid);
+    prm.cs = 0;
+  }
+  e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], prm);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace
@@ -857,6 +1049,8 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   prm.nk = q.nk; prm.nv = q.nv; prm.total_units = q.total_units;
   prm.qk_scale = kLog2e / sqrtf((float)dh);
   prm.pos = a.pos; prm.view = a.view; prm.rank = a.rank;
+  prm.k_cache = static_cast<const __nv_bfloat16*>(a.k_cache);
+  prm.v_cache = static_cast<const __nv_bfloat16*>(a.v_cache);
   prm.out = static_cast<__nv_bfloat16*>(a.out);
   prm.status = a.status;
   prm.partials = static_cast<float*>(a.ws);

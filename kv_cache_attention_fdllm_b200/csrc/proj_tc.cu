@@ -50,12 +50,6 @@ constexpr int kPitch = kChunk + 1;  // staging pitch (floats)
 constexpr int kMaxBN = 256;
 constexpr uint32_t kASubBytes = kBM * kSub * 2;  // 16 KB
 
-__device__ __forceinline__ void grid_dep_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void grid_dep_launch() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
 
 struct ProjTcParams {
   int M, F, D, E, N, H, dh, rows_per_seq, S_max, verify;
@@ -102,7 +96,7 @@ __global__ void __launch_bounds__(128) proj_prep_kernel(const __nv_bfloat16* __r
                                                         int dh, double log2_base,
                                                         __nv_bfloat16* __restrict__ xq,
                                                         float2* __restrict__ rope_tab) {
-  grid_dep_launch();
+  tc::griddep_launch_dependents();
   const int m = blockIdx.x;
   const int ps = idx[m];
   const bool ok = ps >= 0 && ps < N;
@@ -171,6 +165,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the attention kernel that follows may start its prologue on SMs this grid
+  // leaves; it reads nothing of ours before its own grid-dependency wait
+  tc::griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -196,7 +193,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           tc::tma_load_2d(a_s + q * kASubBytes, &tm_w, &full[i], (sb0 + q) * kSub,
                           (tile / p.n_tt) * kBM, pol_w);
       }
-      grid_dep_wait();
+      tc::griddep_wait();
       tile = tile_begin;
       ks = ks_begin;
       for (int i = 0; i < pre; ++i) {
@@ -271,7 +268,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    grid_dep_wait();  // the RoPE table comes from the prep kernel
+    tc::griddep_wait();  // the RoPE table comes from the prep kernel
     const int etid = tid - 64;
     const int quarter = warp & 3;
     const int f_loc = quarter * 32 + lane;
