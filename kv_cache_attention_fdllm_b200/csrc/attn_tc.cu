@@ -170,11 +170,13 @@ struct Smem {
   static constexpr uint32_t kPBufBytes = (kPBytes + 1023) / 1024 * 1024;  // one of two P buffers
 };
 
-// Softmax threads: NQ/16 groups of 4 warps; a thread owns one key (one dh row)
-// and 16 query columns.
+// Softmax threads: NQ/kCols groups of 4 warps; a thread owns one key (one dh
+// row) and kCols query columns (16, or 32 at NQ = 64: 256 threads whose
+// registers hold a tile's 32 scores without spilling).
 template <int NQ>
 struct Threads {
-  static constexpr int kSmx = 8 * NQ;
+  static constexpr int kCols = NQ == 64 ? 32 : 16;
+  static constexpr int kSmx = 128 * NQ / kCols;
   static constexpr int kAll = 64 + kSmx;
 };
 
@@ -427,10 +429,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    // NQ/16 groups of 4 warps: the warps that share a TMEM lane quarter split
+    // NQ/NQH groups of 4 warps: the warps that share a TMEM lane quarter split
     // the query columns, so a thread owns one key (later one dh row) and the
-    // 16 columns [c0, c0 + 16).
-    constexpr int NQH = 16;
+    // NQH columns [c0, c0 + NQH).
+    constexpr int NQH = Threads<NQ>::kCols;
     const int st = tid - 64;                 // 0..kSmx-1
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;        // column group
