@@ -135,6 +135,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   int* last_flag = abort_flag + 1;
   int* tok_slot = reinterpret_cast<int*>(misc + 256);  // -1: skip k, v
   int* tok_flag = tok_slot + kMaxBN;                   // bit0: q valid, bit1: side buffer
+  int* tok_b = tok_flag + kMaxBN;                      // sequence of the token
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -273,6 +274,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     const int quarter = warp & 3;
     const int f_loc = quarter * 32 + lane;
     const int half = p.dh >> 1;
+    const int dh_log2 = p.dh == 128 ? 7 : 6;  // dh is 64 or 128
     float* my_parts = p.partials + (size_t)c * 2 * BN * kBM;
     int j = 0;
     for (long long u = u_begin; u < u_end; ++j) {
@@ -306,6 +308,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         }
         tok_slot[n] = slot;
         tok_flag[n] = flag;
+        tok_b[n] = m < p.M ? m / p.rows_per_seq : 0;
       }
 
       // after a timeout every later wait returns at once: keep going so that all
@@ -395,8 +398,10 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             const int f0 = g * 8;
             const int fg = ft * kBM + f0;
             if (fg >= p.F) continue;
-            const int blk = fg / p.E, rem = fg % p.E;
-            const int h = rem / p.dh, j0 = rem % p.dh;
+            // no integer division: F = 3E and dh is 64 or 128
+            const int blk = fg >= 2 * p.E ? 2 : (fg >= p.E ? 1 : 0);
+            const int rem = fg - blk * p.E;
+            const int h = rem >> dh_log2, j0 = rem & (p.dh - 1);
             const int slot = tok_slot[cc + n], flag = tok_flag[cc + n];
             if (blk != 0 && slot < 0) continue;
             float o[8];
@@ -431,8 +436,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
               __nv_bfloat16* base = (blk == 1) ? (side ? p.k_side : p.k_cache)
                                                : (side ? p.v_side : p.v_cache);
               const int nslots = side ? p.S_max : p.N;
-              const int b = m / p.rows_per_seq;
-              dst = base + (((size_t)b * p.H + h) * nslots + slot) * p.dh + j0;
+              dst = base + (((size_t)tok_b[cc + n] * p.H + h) * nslots + slot) * p.dh + j0;
             }
             *reinterpret_cast<uint4*>(dst) = pk;
           }
@@ -473,7 +477,7 @@ ProjPlan plan(int M, int D, int H, int dh, int num_sms) {
   q.n_ft = (F + kBM - 1) / kBM;
   q.tiles = q.n_ft * q.n_tt;
   q.nsub_total = D / kSub;
-  const size_t fixed = 1024 /*align*/ + (size_t)kBM * kPitch * 4 + 256 + 2 * kMaxBN * 4;
+  const size_t fixed = 1024 /*align*/ + (size_t)kBM * kPitch * 4 + 256 + 3 * kMaxBN * 4;
   // the widest k-step (most contiguous bytes per W row) that keeps two stages
   const int cand[3] = {4, 2, 1};
   for (int i = 0; i < 3; ++i) {
