@@ -43,8 +43,8 @@ namespace {
 
 constexpr int kBM = 128;            // W rows (features) per tile = MMA M
 constexpr int kSub = 64;            // bf16 K elements per sub-block = one 128-byte swizzle row
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
+constexpr int kThreads = 320;
+constexpr int kEpiThreads = 256;    // two warps per TMEM lane quarter
 constexpr int kChunk = 32;          // tokens per epilogue pass
 constexpr int kPitch = kChunk + 1;  // staging pitch (floats)
 constexpr int kMaxBN = 256;
@@ -146,8 +146,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   const int tile_begin = (int)(u_begin / p.nks);
   const int ks_begin = (int)(u_begin - (long long)tile_begin * p.nks);
 
+  // two accumulators of BN columns; a chunk load never reaches past them
   uint32_t ncols = 32;
-  while ((int)ncols < 2 * BN) ncols <<= 1;
+  while ((int)ncols < 2 * BN || (int)ncols < BN + kChunk) ncols <<= 1;
 
   if (tid == 0) {
     for (int s = 0; s < p.nstage; ++s) {
@@ -273,6 +274,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     const int etid = tid - 64;
     const int quarter = warp & 3;
     const int f_loc = quarter * 32 + lane;
+    const int n_half = ((warp - 2) >> 2) * (kChunk / 2);  // this warp's 16 tokens of a chunk
     const int half = p.dh >> 1;
     const int dh_log2 = p.dh == 128 ? 7 : 6;  // dh is 64 or 128
     float* my_parts = p.partials + (size_t)c * 2 * BN * kBM;
@@ -323,13 +325,12 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         // partial tile: store it, free the accumulator, and see who is last
         const int slot = (j == 0) ? 0 : 1;
         float* dst = my_parts + (size_t)slot * BN * kBM;
-        for (int cc = 0; cc < BN; cc += kChunk) {
-          float v[kChunk];
-          tc::tmem_ld32(t_acc + cc, v);
+        for (int cc = n_half; cc < BN; cc += kChunk) {
+          float v[kChunk / 2];
+          tc::tmem_ld16(t_acc + cc, v);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int n = 0; n < kChunk; ++n)
-            if (cc + n < BN) dst[(size_t)(cc + n) * kBM + f_loc] = v[n];
+          for (int n = 0; n < kChunk / 2; ++n) dst[(size_t)(cc + n) * kBM + f_loc] = v[n];
         }
         tc::tc_fence_before();
         __syncwarp();
@@ -354,26 +355,31 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         }
         for (int cc = 0; cc < BN; cc += kChunk) {
           if (whole) {
-            float v[kChunk];
-            tc::tmem_ld32(t_acc + cc, v);
-            tc::tmem_wait_ld();
+            // BN is a multiple of 16: a warp's 16 columns are all in the tile or none
+            if (cc + n_half < BN) {
+              float v[kChunk / 2];
+              tc::tmem_ld16(t_acc + cc + n_half, v);
+              tc::tmem_wait_ld();
 #pragma unroll
-            for (int n = 0; n < kChunk; ++n) staging[f_loc * kPitch + n] = v[n];
+              for (int n = 0; n < kChunk / 2; ++n) staging[f_loc * kPitch + n_half + n] = v[n];
+            }
           } else {
             // sum the partials of every contributor in k order; a thread adds
-            // 4 consecutive features of 8 tokens with 16-byte loads
-            float4 acc[8];
+            // 4 consecutive features of 4 tokens with 16-byte loads
+            constexpr int kTok = kChunk * (kBM / 4) / kEpiThreads;  // 4
+            constexpr int kStride = kEpiThreads / (kBM / 4);        // 8
+            float4 acc[kTok];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = 0; i < kTok; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
             const int f4 = (etid & 31) * 4;
-            const int nb = etid >> 5;  // tokens nb, nb + 4, ...
+            const int nb = etid >> 5;  // tokens nb, nb + 8, ...
             for (int cb = c_first; cb <= c_last; ++cb) {
               // slot 0 when the tile is cb's first: unit_lo(cb) >= tu0
               const int sl = (p.total_units * cb >= tu0 * (long long)G) ? 0 : 1;
               const float* ps = p.partials + ((size_t)cb * 2 + sl) * BN * kBM;
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const int n = cc + nb + 4 * i;
+              for (int i = 0; i < kTok; ++i) {
+                const int n = cc + nb + kStride * i;
                 if (n < BN) {
                   const float4 t = __ldcg(reinterpret_cast<const float4*>(ps + (size_t)n * kBM + f4));
                   acc[i].x += t.x; acc[i].y += t.y; acc[i].z += t.z; acc[i].w += t.w;
@@ -381,8 +387,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
               }
             }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int n = nb + 4 * i;
+            for (int i = 0; i < kTok; ++i) {
+              const int n = nb + kStride * i;
               staging[(f4 + 0) * kPitch + n] = acc[i].x;
               staging[(f4 + 1) * kPitch + n] = acc[i].y;
               staging[(f4 + 2) * kPitch + n] = acc[i].z;
