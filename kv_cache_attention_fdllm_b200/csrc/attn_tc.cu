@@ -49,7 +49,7 @@ constexpr int kL2PrefetchTiles = 4;  // cache tiles per CTA warmed in L2 before 
 
 struct AttnTcParams {
   int B, N, H, rows, S_max, causal;
-  int n_qc, n_cache_tiles, n_side_tiles, tpi, nk, nv;
+  int n_qc, n_cache_tiles, n_side_tiles, tpi, nk, nv, nqbuf;
   long long total_units;
   float qk_scale;  // log2(e) / sqrt(dh)
   const int32_t* pos;
@@ -194,7 +194,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint8_t* k_ring = smem;
   uint8_t* v_ring = smem + NK * L::kTileBytes;
   uint8_t* q_buf = v_ring + NV * L::kTileBytes;
-  uint8_t* p_buf = q_buf + 2 * L::kQBytes;  // 1024-aligned (kQBytes is a multiple of 1024)
+  uint8_t* p_buf = q_buf + p.nqbuf * L::kQBytes;  // 1024-aligned (kQBytes is a multiple of 1024)
   uint8_t* misc = p_buf + 2 * L::kPBufBytes;
   uint64_t* k_full = reinterpret_cast<uint64_t*>(misc);
   uint64_t* k_empty = k_full + 8;
@@ -899,10 +899,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 }
 
 struct AttnPlan {
-  int NQ, n_qc, nct, nst, tpi, nk, nv, grid;  // grid: stream-K grid
-  int cs;                                      // cluster size wanted (0: stream-K)
+  int NQ, n_qc, nct, nst, tpi, nk, nv, grid;  // stream-K: rings, grid
+  int cs, nk_cl, nv_cl;                        // cluster size wanted (0: stream-K), its rings
   long long items, total_units;
-  size_t smem_bytes, partial_bytes, counter_bytes;
+  size_t smem_bytes, smem_cl, partial_bytes, counter_bytes;
 };
 
 constexpr size_t kSmemBudget = 227 * 1024;
@@ -929,14 +929,23 @@ AttnPlan plan(int B, int N, int H, int dh, int rows, int S_max, int verify, int 
   const size_t tile = boxes * 16384;
   const size_t qbytes = boxes * q.NQ * 128;
   const size_t pbytes = 2 * (((size_t)kKT * q.NQ * 2 + 1023) / 1024 * 1024);
-  const size_t fixed = 1024 + 2 * qbytes + pbytes + 4096 + 3 * kMaxRows * 4;
-  // K and V tiles share what shared memory is left; K gets the odd one
-  int tiles = (int)((kSmemBudget - fixed) / tile);
-  if (tiles > 16) tiles = 16;
-  q.nv = tiles / 2;
-  q.nk = tiles - q.nv;
-  if (q.nk > 8) q.nk = 8;
-  q.smem_bytes = fixed + (size_t)(q.nk + q.nv) * tile;
+  // misc: barriers and softmax scratch, then the verify tables (or, without
+  // them, the [8][NQ] merge weights of the stream-K path)
+  const size_t misc = 4096 + (verify ? 3 * kMaxRows * 4 : 8 * 64 * 4);
+  // K and V tiles share what shared memory is left.  A V tile is held from its
+  // load until its PV is done, longer than a K tile, so V gets the odd one.
+  // Cluster mode runs one item per CTA and needs one Q buffer, not two.
+  auto rings = [&](int nqbuf, int& nk, int& nv) -> size_t {
+    const size_t fixed = 1024 + nqbuf * qbytes + pbytes + misc;
+    int tiles = (int)((kSmemBudget - fixed) / tile);
+    if (tiles > 16) tiles = 16;
+    nv = (tiles + 1) / 2;
+    nk = tiles - nv;
+    if (nv > 8) nv = 8;
+    return fixed + (size_t)(nk + nv) * tile;
+  };
+  q.smem_bytes = rings(2, q.nk, q.nv);
+  q.smem_cl = rings(1, q.nk_cl, q.nv_cl);
   q.partial_bytes = align_up((size_t)q.grid * 2 * ((size_t)q.NQ * dh + 2 * q.NQ) * sizeof(float), 256);
   q.counter_bytes = align_up((size_t)q.items * sizeof(unsigned), 256);
   return q;
@@ -972,15 +981,15 @@ template <int NQ, int DH, bool VERIFY>
 cudaError_t launch_t(const AttnArgs& a, const AttnPlan& q, AttnTcParams prm, const CUtensorMap* maps,
                      cudaStream_t stream) {
   auto kern = attn_tc_kernel<NQ, DH, VERIFY>;
+  const size_t smem_max = q.smem_bytes > q.smem_cl ? q.smem_bytes : q.smem_cl;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)q.smem_bytes);
+                                       (int)smem_max);
   if (e != cudaSuccess) return e;
   // cluster mode only when every item's cluster fits in one wave
   int cs = q.cs;
-  while (cs >= 2 && max_clusters<NQ, DH, VERIFY>(cs, q.smem_bytes) < q.items) --cs;
+  while (cs >= 2 && max_clusters<NQ, DH, VERIFY>(cs, q.smem_cl) < q.items) --cs;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(Threads<NQ>::kAll);
-  cfg.dynamicSmemBytes = q.smem_bytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -994,10 +1003,18 @@ cudaError_t launch_t(const AttnArgs& a, const AttnPlan& q, AttnTcParams prm, con
     attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
     cfg.gridDim = dim3((unsigned)(q.items * cs));
+    cfg.dynamicSmemBytes = q.smem_cl;
     prm.cs = cs;
+    prm.nk = q.nk_cl;
+    prm.nv = q.nv_cl;
+    prm.nqbuf = 1;
   } else {
     cfg.gridDim = dim3(q.grid);
+    cfg.dynamicSmemBytes = q.smem_bytes;
     prm.cs = 0;
+    prm.nk = q.nk;
+    prm.nv = q.nv;
+    prm.nqbuf = 2;
   }
   e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], prm);
   count_launches(1);
@@ -1048,7 +1065,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   prm.B = a.B; prm.N = a.N; prm.H = a.H; prm.rows = a.rows_per_seq; prm.S_max = a.S_max;
   prm.causal = a.causal_cross;
   prm.n_qc = q.n_qc; prm.n_cache_tiles = q.nct; prm.n_side_tiles = q.nst; prm.tpi = q.tpi;
-  prm.nk = q.nk; prm.nv = q.nv; prm.total_units = q.total_units;
+  prm.total_units = q.total_units;
   prm.qk_scale = kLog2e / sqrtf((float)dh);
   prm.pos = a.pos; prm.view = a.view; prm.rank = a.rank;
   prm.k_cache = static_cast<const __nv_bfloat16*>(a.k_cache);
