@@ -10,11 +10,9 @@
 // tokens] = W_tile[128 x K] * X[BN x K]^T, so W rows fill the MMA's M = 128 and
 // the gathered tokens are its N (16..256).
 //
-// Two kernels, the second launched as a programmatic dependent of the first:
-//   proj_prep    one CTA per row: packs x[Q] into the workspace (fused step;
-//                verify rows arrive packed) and tabulates the RoPE cos/sin of
-//                the row's position, so the epilogue does no transcendental
-//                math.  It lets the projection start at once.
+// Fused step: two kernels, the second launched as a programmatic dependent of
+// the first (verify rows arrive packed, so the verify pass runs the second only):
+//   proj_prep    one CTA per row: packs x[Q] into the workspace.
 //   proj_tc      persistent stream-K GEMM.  Its W loads do not depend on the
 //                prep kernel and are issued before the grid-dependency wait.
 //
@@ -30,8 +28,11 @@
 //   warp 0      TMA producer: W boxes [64 x 128] and X boxes [64 x BN]
 //   warp 1      TMEM allocation; lane 0 issues tcgen05.mma into one of two
 //               TMEM accumulators (the epilogue drains the other)
-//   warps 2-5   epilogue: TMEM (or the summed partials) -> shared memory ->
-//               RoPE on the q and k heads -> 16-byte stores of q, k, v rows
+//   warps 2-9   epilogue, two warps per TMEM lane quarter: TMEM (or the summed
+//               partials) -> shared memory -> RoPE on the q and k heads (cos
+//               and sin computed in place: the angle reduced modulo 2 pi in
+//               double, then the fast single-precision sine and cosine) ->
+//               16-byte stores of q, k, v rows
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -49,6 +50,8 @@ constexpr int kChunk = 32;          // tokens per epilogue pass
 constexpr int kPitch = kChunk + 1;  // staging pitch (floats)
 constexpr int kMaxBN = 256;
 constexpr uint32_t kASubBytes = kBM * kSub * 2;  // 16 KB
+constexpr double kTwoPi = 6.283185307179586476925286766559;
+constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
 
 
 struct ProjTcParams {
@@ -57,7 +60,7 @@ struct ProjTcParams {
   long long total_units;
   const int32_t* idx;
   const int8_t* view;
-  const float2* rope_tab;  // [M][dh/2] (cos, sin) of the row's position
+  double log2_base;        // log2 of the RoPE base
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
   __nv_bfloat16* k_side;
@@ -88,31 +91,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// One CTA per projection row m: xq[m] = x[b, q_idx[m]] (fused step; zeros when
-// the index is out of range) and rope_tab[m][j] = (cos, sin)(pos * theta_j).
+// One CTA per projection row m of the fused step: xq[m] = x[b, q_idx[m]] (zeros
+// when the index is out of range).
 __global__ void __launch_bounds__(128) proj_prep_kernel(const __nv_bfloat16* __restrict__ x,
                                                         const int32_t* __restrict__ idx, int N,
-                                                        int D, int rows_per_seq, int verify,
-                                                        int dh, double log2_base,
-                                                        __nv_bfloat16* __restrict__ xq,
-                                                        float2* __restrict__ rope_tab) {
+                                                        int D, int rows_per_seq,
+                                                        __nv_bfloat16* __restrict__ xq) {
   tc::griddep_launch_dependents();
   const int m = blockIdx.x;
   const int ps = idx[m];
   const bool ok = ps >= 0 && ps < N;
-  if (!verify) {
-    const int b = m / rows_per_seq;
-    const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)b * N + (ok ? ps : 0)) * D);
-    uint4* dst = reinterpret_cast<uint4*>(xq + (size_t)m * D);
-    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    for (int i = threadIdx.x; i < D / 8; i += blockDim.x) dst[i] = ok ? __ldg(src + i) : zero;
-  }
-  const int half = dh / 2;
-  for (int j = threadIdx.x; j < half; j += blockDim.x) {
-    float c, s;
-    rope_cos_sin(ok ? ps : 0, rope_inv_freq(j, dh, log2_base), &c, &s);
-    rope_tab[(size_t)m * half + j] = make_float2(c, s);
-  }
+  const int b = m / rows_per_seq;
+  const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)b * N + (ok ? ps : 0)) * D);
+  uint4* dst = reinterpret_cast<uint4*>(xq + (size_t)m * D);
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = threadIdx.x; i < D / 8; i += blockDim.x) dst[i] = ok ? __ldg(src + i) : zero;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -136,6 +129,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   int* tok_slot = reinterpret_cast<int*>(misc + 256);  // -1: skip k, v
   int* tok_flag = tok_slot + kMaxBN;                   // bit0: q valid, bit1: side buffer
   int* tok_b = tok_flag + kMaxBN;                      // sequence of the token
+  int* tok_pos = tok_b + kMaxBN;                       // RoPE position (0 for a skipped row)
+  double* theta = reinterpret_cast<double*>(tok_pos + kMaxBN);  // [dh/2] RoPE frequencies
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -270,8 +265,13 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    tc::griddep_wait();  // the RoPE table comes from the prep kernel
+    tc::griddep_wait();
     const int etid = tid - 64;
+    // theta_j = base^(-2j/dh), in double: the angle pos * theta_j is reduced
+    // modulo 2 pi in double before the single-precision sine and cosine
+    for (int jj = etid; jj < (p.dh >> 1); jj += kEpiThreads)
+      theta[jj] = exp2(-(2.0 * (double)jj / (double)p.dh) * p.log2_base);
+    tc::named_bar_sync(1, kEpiThreads);
     const int quarter = warp & 3;
     const int f_loc = quarter * 32 + lane;
     const int n_half = ((warp - 2) >> 2) * (kChunk / 2);  // this warp's 16 tokens of a chunk
@@ -311,6 +311,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         tok_slot[n] = slot;
         tok_flag[n] = flag;
         tok_b[n] = m < p.M ? m / p.rows_per_seq : 0;
+        tok_pos[n] = (flag & 1) ? p.idx[m] : 0;
       }
 
       // after a timeout every later wait returns at once: keep going so that all
@@ -420,13 +421,18 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             } else {
               const bool lo = j0 < half;
               const int pf = lo ? f0 + half : f0 - half;
-              const float2* tab = p.rope_tab + (size_t)m * half + (lo ? j0 : j0 - half);
+              const double* th = theta + (lo ? j0 : j0 - half);
+              const double pos = (double)tok_pos[cc + n];
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
                 const float x = staging[(f0 + i) * kPitch + n];
                 const float xp = staging[(pf + i) * kPitch + n];
-                const float2 cs = __ldg(tab + i);
-                o[i] = lo ? (x * cs.x - xp * cs.y) : (xp * cs.y + x * cs.x);
+                // angle mod 2 pi in double, then the fast sine/cosine on [-pi, pi]
+                const double ang = pos * th[i];
+                const double k = rint(ang * kInvTwoPi);
+                float sn, cs;
+                __sincosf((float)fma(-k, kTwoPi, ang), &sn, &cs);
+                o[i] = lo ? (x * cs - xp * sn) : (xp * sn + x * cs);
               }
             }
             uint4 pk;
@@ -469,7 +475,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
 struct ProjPlan {
   int BN, n_tt, n_ft, tiles, nks, subs, nsub_total, nstage, grid;
   long long total_units;
-  size_t smem_bytes, partial_bytes, counter_bytes, xq_bytes, tab_bytes;
+  size_t smem_bytes, partial_bytes, counter_bytes, xq_bytes;
 };
 
 constexpr size_t kSmemBudget = 227 * 1024;
@@ -483,7 +489,7 @@ ProjPlan plan(int M, int D, int H, int dh, int num_sms) {
   q.n_ft = (F + kBM - 1) / kBM;
   q.tiles = q.n_ft * q.n_tt;
   q.nsub_total = D / kSub;
-  const size_t fixed = 1024 /*align*/ + (size_t)kBM * kPitch * 4 + 256 + 3 * kMaxBN * 4;
+  const size_t fixed = 1024 /*align*/ + (size_t)kBM * kPitch * 4 + 256 + 4 * kMaxBN * 4 + 64 * 8;
   // the widest k-step (most contiguous bytes per W row) that keeps two stages
   const int cand[3] = {4, 2, 1};
   for (int i = 0; i < 3; ++i) {
@@ -506,7 +512,6 @@ ProjPlan plan(int M, int D, int H, int dh, int num_sms) {
   q.partial_bytes = align_up((size_t)q.grid * 2 * q.BN * kBM * sizeof(float), 256);
   q.counter_bytes = align_up((size_t)q.tiles * sizeof(unsigned), 256);
   q.xq_bytes = align_up((size_t)M * D * 2, 256);
-  q.tab_bytes = align_up((size_t)M * (dh / 2) * sizeof(float2), 256);
   return q;
 }
 
@@ -515,7 +520,7 @@ ProjPlan plan(int M, int D, int H, int dh, int num_sms) {
 size_t proj_tc_workspace_bytes(int M, int D, int H, int dh, int num_sms) {
   if (M <= 0) return 256;
   const ProjPlan q = plan(M, D, H, dh, num_sms);
-  return q.partial_bytes + q.counter_bytes + q.xq_bytes + q.tab_bytes;
+  return q.partial_bytes + q.counter_bytes + q.xq_bytes;
 }
 
 cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream) {
@@ -523,11 +528,10 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream) {
   if (M == 0) return cudaSuccess;
   const int E = a.H * a.dh, F = 3 * E;
   const ProjPlan q = plan(M, a.D, a.H, a.dh, device_sm_count());
-  if (q.partial_bytes + q.counter_bytes + q.xq_bytes + q.tab_bytes > a.ws_bytes)
+  if (q.partial_bytes + q.counter_bytes + q.xq_bytes > a.ws_bytes)
     return cudaErrorInvalidValue;
   char* ws = static_cast<char*>(a.ws);
   __nv_bfloat16* xq = reinterpret_cast<__nv_bfloat16*>(ws + q.partial_bytes + q.counter_bytes);
-  float2* tab = reinterpret_cast<float2*>(ws + q.partial_bytes + q.counter_bytes + q.xq_bytes);
 
   CUtensorMap tm_w, tm_x;
   {
@@ -553,7 +557,7 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream) {
   p.rows_per_seq = a.rows_per_seq; p.S_max = a.S_max; p.verify = a.verify;
   p.BN = q.BN; p.n_tt = q.n_tt; p.tiles = q.tiles; p.nks = q.nks; p.subs = q.subs;
   p.nsub_total = q.nsub_total; p.nstage = q.nstage; p.total_units = q.total_units;
-  p.idx = a.idx; p.view = a.view; p.rope_tab = tab;
+  p.idx = a.idx; p.view = a.view; p.log2_base = a.log2_base;
   p.k_cache = static_cast<__nv_bfloat16*>(a.k_cache);
   p.v_cache = static_cast<__nv_bfloat16*>(a.v_cache);
   p.k_side = static_cast<__nv_bfloat16*>(a.k_side);
@@ -563,12 +567,15 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream) {
   p.partials = reinterpret_cast<float*>(ws);
   p.tile_cnt = reinterpret_cast<unsigned*>(ws + q.partial_bytes);
 
-  proj_prep_kernel<<<M, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.x), a.idx, a.N,
-                                          a.D, a.rows_per_seq, a.verify, a.dh, a.log2_base, xq,
-                                          tab);
-  count_launches(1);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
+  if (!a.verify) {
+    // the fused step gathers x[Q] into a packed operand; verify rows arrive packed
+    proj_prep_kernel<<<M, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.x), a.idx, a.N,
+                                            a.D, a.rows_per_seq, xq);
+    count_launches(1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
 
   e = cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)q.smem_bytes);
