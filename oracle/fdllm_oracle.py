@@ -25,6 +25,9 @@ What is computed (each function states its passage):
   * accept       - top-1 / confidence, the epsilon split into D_t / S_t and the
                    gamma prefix acceptance ([review], "Flash-Verify", sec. 2.3
                    and the worked example).
+  * attention_mass, track_select - the tracked set of the next step ([review],
+                   "How It Works", Step 1: Cache selection): the decoded slots
+                   most attended by the masked queries.
 
 Everything is computed in float64 from the exactly upcast stored inputs.  The
 k,v written into the cache are rounded once to the storage dtype, and the
@@ -309,3 +312,55 @@ def accept(logits, kind, ref_tok, rank, eps, gamma):
                 flags[b, r] |= FLAG_ACCEPT
                 n_accept[b] += 1
     return top1, conf, flags, n_accept
+
+
+# ----------------------------------------------------------------------------
+# tracked-set selection
+
+
+def attention_mass(x, q_idx, w_qkv, rope_base, k_cache2, H, dh, masked_row):
+    """Attention mass of every cache slot ([review], "How It Works", Step 1:
+    Cache selection, which ranks decoded tokens by how much the masked queries
+    attend to them).
+
+    Reading: a[b, j] = sum over the masked-query rows i of Q (masked_row[b, i]
+    != 0) and over the heads h of softmax_j(q_ih . K'_hj / sqrt(dh)), the
+    softmax taken over all N slots of the cache K' the step left (k_cache2,
+    after the write at Q), exactly the probabilities of the draft pass.  q is
+    the step's query: x[b, Q] projected and rotated at Q.  Returns [B, N]."""
+    B, nq = q_idx.shape
+    N = k_cache2.shape[2]
+    a = np.zeros((B, N))
+    for b in range(B):
+        Q = np.asarray(q_idx[b], dtype=np.int64)
+        rows = np.nonzero(np.asarray(masked_row[b]) != 0)[0]
+        if rows.size == 0:
+            continue
+        q, _, _ = project_qkv(x[b, Q[rows]], w_qkv, H, dh)
+        q = rope(q, Q[rows], rope_base)
+        for h in range(H):
+            s = (q[:, h] @ k_cache2[b, h].T) / np.sqrt(dh)
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            p = p / p.sum(axis=1, keepdims=True)
+            a[b] += p.sum(axis=0)
+    return a
+
+
+def track_select(a, candidate, beta_t):
+    """The next tracked set T ([review], "How It Works", Step 1: Cache
+    selection): the beta_t candidate slots with the largest attention mass.
+
+    candidate[b, j] != 0 marks a decoded slot.  The positions decoded in this
+    step are candidates like the earlier ones (the page includes the newly
+    resolved positions before ranking and keeps |T| at beta_t).  Order: mass
+    descending, equal mass to the lower slot.  With fewer candidates than
+    beta_t the tail is -1.  Returns int64 [B, beta_t]."""
+    B, N = a.shape
+    out = np.full((B, beta_t), -1, dtype=np.int64)
+    for b in range(B):
+        cand = [j for j in range(N) if candidate[b, j] != 0]
+        cand.sort(key=lambda j: (-a[b, j], j))
+        for t, j in enumerate(cand[:beta_t]):
+            out[b, t] = j
+    return out

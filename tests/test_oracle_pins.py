@@ -359,3 +359,94 @@ def test_accept_ties_uniform_and_tv_bound():
         order = np.argsort(rank[0])
         seq = acc[order]
         assert not np.any(seq[1:] & ~seq[:-1])
+
+
+# ----------------------------------------------------------------------------
+# tracked-set selection ([review], "How It Works", Step 1: Cache selection)
+
+
+def _mass_case(seed, B=2, N=40, D=64, H=3, dh=64, nq=6):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((B, N, D))
+    w = rng.standard_normal((3 * H * dh, D)) / np.sqrt(D)
+    K = rng.standard_normal((B, H, N, dh))
+    V = rng.standard_normal((B, H, N, dh))
+    q_idx = np.stack([rng.choice(N, nq, replace=False) for _ in range(B)])
+    masked = (rng.random((B, nq)) < 0.5).astype(np.int8)
+    masked[:, 0] = 1
+    K2, V2, _ = O.fused_step(x, q_idx, w, 10000.0, K, V, H, dh, "f64")
+    return x, q_idx, w, K2, masked, H, dh
+
+
+def test_attention_mass_is_sdpa_probabilities():
+    """With V = the identity, torch's scaled-dot-product attention returns the
+    softmax probabilities themselves; summed over the masked rows and heads
+    they must equal the oracle's attention mass (catches a wrong scale, a
+    softmax over the wrong axis or a transposed operand)."""
+    x, q_idx, w, K2, masked, H, dh = _mass_case(21)
+    a = O.attention_mass(x, q_idx, w, 10000.0, K2, H, dh, masked)
+    B, N = a.shape
+    for b in range(B):
+        rows = np.nonzero(masked[b])[0]
+        Q = q_idx[b][rows]
+        q, _, _ = O.project_qkv(x[b, Q], w, H, dh)
+        q = O.rope(q, Q, 10000.0)
+        ref = np.zeros(N)
+        eye = torch.eye(N, dtype=torch.float64)
+        for h in range(H):
+            p = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q[:, h])[None], torch.from_numpy(K2[b, h])[None], eye[None])[0]
+            ref += p.numpy().sum(axis=0)
+        np.testing.assert_allclose(a[b], ref, rtol=1e-12, atol=1e-14)
+
+
+def test_attention_mass_closed_forms():
+    """Each masked row and head spreads probability 1 over the N slots: the
+    mass sums to (masked rows) x H.  Equal keys give every slot the same
+    share; no masked row gives no mass."""
+    x, q_idx, w, K2, masked, H, dh = _mass_case(22)
+    a = O.attention_mass(x, q_idx, w, 10000.0, K2, H, dh, masked)
+    np.testing.assert_allclose(a.sum(axis=1), masked.sum(axis=1) * H, rtol=1e-12)
+    Kc = np.broadcast_to(K2[:, :, :1, :], K2.shape).copy()
+    a_eq = O.attention_mass(x, q_idx, w, 10000.0, Kc, H, dh, masked)
+    N = K2.shape[2]
+    np.testing.assert_allclose(a_eq, (masked.sum(axis=1) * H / N)[:, None] * np.ones((1, N)),
+                               rtol=1e-12)
+    assert not O.attention_mass(x, q_idx, w, 10000.0, K2, H, dh, np.zeros_like(masked)).any()
+
+
+def test_track_select_order_ties_and_padding():
+    a = np.array([[0.5, 2.0, 2.0, 0.1, 3.0, 2.0]])
+    cand = np.array([[1, 1, 1, 1, 0, 1]])
+    # slot 4 has the most mass but is not decoded; 1, 2, 5 tie: lower slot first
+    assert O.track_select(a, cand, 4).tolist() == [[1, 2, 5, 0]]
+    assert O.track_select(a, cand, 7).tolist() == [[1, 2, 5, 0, 3, -1, -1]]
+    assert O.track_select(a, np.zeros_like(cand), 2).tolist() == [[-1, -1]]
+
+
+def test_track_select_worked_example_rule():
+    """The review's example: [BOS] + 4 masks, slot 0 decoded before the step,
+    Q = {1, 2} (the front beta_m = 2 masks), both resolved by the step, beta_t
+    = 1.  The resolved slots join the ranking, so T keeps exactly one slot, and
+    it is the slot the masked queries attend to most.  The cache is built so
+    that one key dominates every score (closed form: it takes all the mass)."""
+    H, dh, N, D = 2, 64, 5, 64
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((1, N, D))
+    w = rng.standard_normal((3 * H * dh, D)) / np.sqrt(D)
+    q_idx = np.array([[1, 2]])
+    masked = np.array([[1, 1]], dtype=np.int8)
+    cand = np.array([[1, 1, 1, 0, 0]])  # slot 0 earlier; 1, 2 resolved now
+    for target in (0, 2):
+        K = rng.standard_normal((1, H, N, dh)) * 1e-3
+        V = np.zeros((1, H, N, dh))
+        K2, _, _ = O.fused_step(x, q_idx, w, 10000.0, K, V, H, dh, "f64")
+        q, _, _ = O.project_qkv(x[0, q_idx[0]], w, H, dh)
+        q = O.rope(q, q_idx[0], 10000.0)
+        for h in range(H):
+            # a key along the sum of the queries' directions, far above the rest
+            K2[0, h, target] = 400.0 * (q[:, h] / np.linalg.norm(q[:, h], axis=1, keepdims=True)).sum(0)
+            K2[0, h, 1:3] *= 1e-6 if target == 0 else 1.0
+        a = O.attention_mass(x, q_idx, w, 10000.0, K2, H, dh, masked)
+        assert a[0, target] > 0.999 * 2 * H
+        assert O.track_select(a, cand, 1).tolist() == [[target]]
