@@ -19,6 +19,9 @@
  *   fdllm_accept       per-row top-1 and confidence, the epsilon split D_t / S_t
  *                      and the gamma prefix acceptance up to the first mismatch
  *                      ([review] "Flash-Verify", sec. 2.3 and the worked example).
+ *   fdllm_track_select the tracked set of the next step: the decoded slots the
+ *                      masked queries attend to most ([review] "How It Works",
+ *                      Step 1: Cache selection).
  *
  * Conventions shared by every call
  *   - Every pointer argument is a DEVICE pointer owned by the caller, unless
@@ -207,6 +210,36 @@ fdllm_status fdllm_accept_noalloc(int B, int R, int V, const float* logits, cons
                                   const int32_t* ref_tok, const int32_t* rank, float eps,
                                   float gamma, int32_t* top1, float* conf, uint8_t* flags,
                                   int32_t* n_accept, void* stream);
+
+/* Largest tracked-set size fdllm_track_select accepts. */
+#define FDLLM_MAX_BETA_T 1024
+
+/* The tracked set of the next step ([review] "How It Works", Step 1: Cache
+ * selection): the beta_t decoded cache slots that the step's masked queries
+ * attend to most.
+ *   Call it after fdllm_fused_step (or fdllm_qkv_rope_scatter followed by
+ *   fdllm_attend) on the SAME workspace, with the same B, N, H, dh, nq, dtype,
+ *   and before that workspace is used again: it reads the rotated queries and
+ *   the per-row softmax normalisers the step left there.  k_cache is the cache
+ *   as that step left it.
+ *   Attention mass: a[b, j] = sum over the rows i of Q with q_masked[b, i] != 0
+ *   (the masked queries M^{beta_m}) and over the heads h of the step's softmax
+ *   probability p_ihj (taken over all N slots).
+ *   q_masked   int8 [B, nq]    1 = masked-query row, 0 = tracked row
+ *   candidate  int8 [B, N]     1 = decoded slot (the slots decoded in this
+ *                              step included: they are ranked with the rest)
+ *   beta_t     1..FDLLM_MAX_BETA_T
+ *   track      int32 [B, beta_t] out: the candidates with the largest mass,
+ *              mass descending, equal mass to the lower slot; -1 past the
+ *              number of candidates
+ *   mass       float [B, N] out, may be NULL: a[b, j] for every slot
+ *   Deterministic: the heads are summed in order and the selection is exact
+ *   on the fp32 masses.  Returns FDLLM_ERR_UNSUPPORTED for beta_t out of range;
+ *   FDLLM_ERR_WORKSPACE when the workspace is smaller than the fused step's. */
+fdllm_status fdllm_track_select(int B, int N, int H, int dh, int nq, int dtype,
+                                const int8_t* q_masked, const int8_t* candidate,
+                                const void* k_cache, int beta_t, int32_t* track, float* mass,
+                                void* workspace, size_t workspace_bytes, void* stream);
 
 /* Number of kernels this library has launched in this process (a diagnostic
  * counter, incremented on the host at every launch; never reset). */

@@ -15,7 +15,7 @@ from .api import (ERR_BAD_INDEX, ERR_CUDA, ERR_INVALID_ARG, ERR_TIMEOUT, ERR_UNS
                   fdllm_accept_workspace_bytes, fdllm_attend,
                   fdllm_fused_step, fdllm_fused_step_workspace_bytes, fdllm_get_status,
                   fdllm_qkv_rope_scatter, fdllm_verify_attend, fdllm_verify_qkv_rope_scatter,
-                  fdllm_verify_step, fdllm_verify_step_workspace_bytes)
+                  fdllm_track_select, fdllm_verify_step, fdllm_verify_step_workspace_bytes)
 
 from .shard import max_over_ranks, rank_sequences  # noqa: E402
 

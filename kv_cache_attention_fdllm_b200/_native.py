@@ -34,6 +34,8 @@ SIGNATURES = {
                                              _vp, _vp, _vp, _c_size, _vp]),
     "fdllm_accept_noalloc": (_c_int, [_c_int] * 3 + [_vp, _vp, _vp, _vp, _c_float, _c_float,
                                                      _vp, _vp, _vp, _vp, _vp]),
+    "fdllm_track_select": (_c_int, [_c_int] * 6 + [_vp, _vp, _vp, _c_int, _vp, _vp, _vp, _c_size,
+                                                    _vp]),
     "fdllm_launch_count": (ctypes.c_uint64, []),
     "fdllm_get_status": (_c_int, [_vp, _vp]),
 }

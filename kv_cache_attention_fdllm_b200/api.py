@@ -216,6 +216,32 @@ def fdllm_verify_attend(q, pos, view, rank, k_cache, v_cache, k_side, v_side, ou
 
 # ---------------------------------------------------------------- acceptance
 
+def fdllm_track_select(q_masked, candidate, k_cache, track, workspace, mass=None, dtype=None,
+                       stream=None):
+    """The next tracked set from the last fused step on `workspace` (see include/fdllm.h).
+
+    q_masked int8 [B, nq], candidate int8 [B, N], k_cache [B, H, N, dh] as the
+    step left it, track int32 [B, beta_t] (out), mass float32 [B, N] (out, optional)."""
+    _need(q_masked, "q_masked", torch.int8)
+    B, nq = q_masked.shape
+    _need(k_cache, "k_cache")
+    _, H, N, dh = k_cache.shape
+    dev = k_cache.device
+    _need(q_masked, "q_masked", torch.int8, (B, nq), dev)
+    _need(candidate, "candidate", torch.int8, (B, N), dev)
+    _need(track, "track", torch.int32, None, dev)
+    if track.dim() != 2 or track.shape[0] != B:
+        raise ValueError(f"track must be [B, beta_t] with B={B}, got {tuple(track.shape)}")
+    if mass is not None:
+        _need(mass, "mass", torch.float32, (B, N), dev)
+    _need(workspace, "workspace", torch.uint8, None, dev)
+    st = lib().fdllm_track_select(B, N, H, dh, nq, _dtype_code(k_cache), _p(q_masked),
+                                  _p(candidate), _p(k_cache), track.shape[1], _p(track), _p(mass),
+                                  _p(workspace), workspace.numel(), _stream(stream))
+    _check(st, "fdllm_track_select")
+    return track, mass
+
+
 def fdllm_accept(logits, kind, ref_tok, rank, top1, conf, flags, n_accept, workspace, eps=0.9,
                  gamma=0.8, stream=None):
     """Top-1, confidence, epsilon split and gamma prefix acceptance (see include/fdllm.h)."""

@@ -30,13 +30,16 @@ fdllm_status check_shape(int B, int N, int D, int H, int dh, int rows, int dtype
   return FDLLM_OK;
 }
 
-// Workspace layout shared by a full step and its two stage calls:
-//   [header 256 B | q staging | attention scratch | projection scratch]
-// The attention region does not depend on D, so a stage attention call finds
-// it at the same offset whatever D the full step was sized for.
+// Workspace layout shared by a full step, its two stage calls and the
+// tracked-set selection that follows a fused step:
+//   [header 256 B | q staging | lse | selection scratch (fused step only) |
+//    attention scratch | projection scratch]
+// Everything before the projection region is independent of D, so a stage
+// attention call or a selection call finds it at the same offsets whatever D
+// the full step was sized for.
 struct Layout {
-  size_t q_off, attn_off, proj_off, total;
-  size_t proj_bytes, attn_bytes;
+  size_t q_off, lse_off, track_off, attn_off, proj_off, total;
+  size_t track_bytes, proj_bytes, attn_bytes;
 };
 
 Layout step_layout(int B, int N, int D, int H, int dh, int rows, int S_max, int verify,
@@ -45,7 +48,10 @@ Layout step_layout(int B, int N, int D, int H, int dh, int rows, int S_max, int 
   Layout L;
   L.q_off = kWsHeaderBytes;
   const size_t q_bytes = align_up((size_t)B * rows * H * dh * elt_size(dtype), 256);
-  L.attn_off = L.q_off + q_bytes;
+  L.lse_off = L.q_off + q_bytes;
+  L.track_off = L.lse_off + align_up((size_t)B * rows * H * sizeof(float), 256);
+  L.track_bytes = verify ? 0 : align_up(track_workspace_bytes(B, N, H), 256);
+  L.attn_off = L.track_off + L.track_bytes;
   L.attn_bytes =
       align_up(attn_workspace_bytes(B, N, H, dh, rows, S_max, verify, dtype, sms), 256);
   L.proj_off = L.attn_off + L.attn_bytes;
@@ -92,6 +98,7 @@ fdllm_status run_attn(int B, int N, int H, int dh, int rows, int S_max, int veri
   a.verify = verify; a.causal_cross = causal; a.dtype = dtype;
   a.q = q; a.k_cache = k_cache; a.v_cache = v_cache; a.k_side = k_side; a.v_side = v_side;
   a.pos = pos; a.view = view; a.rank = rank; a.out = out;
+  a.lse = reinterpret_cast<float*>(ws_at(ws, L.lse_off));
   a.status = reinterpret_cast<int*>(ws);
   a.ws = ws_at(ws, L.attn_off);
   a.ws_bytes = L.attn_bytes;
@@ -313,6 +320,32 @@ fdllm_status fdllm_accept(int B, int R, int V, const float* logits, const int8_t
   off += align_up((size_t)rows * sizeof(unsigned), 256);
   a.seq_cnt = reinterpret_cast<unsigned*>(ws_at(workspace, off));
   return from_cuda(launch_accept(a, static_cast<cudaStream_t>(stream)));
+}
+
+fdllm_status fdllm_track_select(int B, int N, int H, int dh, int nq, int dtype,
+                                const int8_t* q_masked, const int8_t* candidate,
+                                const void* k_cache, int beta_t, int32_t* track, float* mass,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  fdllm_status st = check_shape(B, N, 64, H, dh, nq, dtype);
+  if (st != FDLLM_OK) return st;
+  if (beta_t < 1 || beta_t > kMaxBetaT) return FDLLM_ERR_UNSUPPORTED;
+  // the regions it reads and uses sit before the D-dependent projection region
+  const Layout L = step_layout(B, N, 64, H, dh, nq, 0, 0, dtype);
+  if ((st = check_ws(workspace, workspace_bytes, L.track_off + L.track_bytes)) != FDLLM_OK)
+    return st;
+  if (B == 0) return FDLLM_OK;
+  if (!all_aligned({q_masked, candidate, k_cache, track})) return FDLLM_ERR_INVALID_ARG;
+  if (mass && !aligned16(mass)) return FDLLM_ERR_INVALID_ARG;
+  TrackArgs a{};
+  a.B = B; a.N = N; a.H = H; a.dh = dh; a.nq = nq; a.dtype = dtype; a.beta_t = beta_t;
+  a.q = ws_at(workspace, L.q_off);
+  a.lse = reinterpret_cast<const float*>(ws_at(workspace, L.lse_off));
+  a.q_masked = q_masked; a.candidate = candidate; a.k_cache = k_cache; a.track = track;
+  a.mass_h = reinterpret_cast<float*>(ws_at(workspace, L.track_off));
+  a.mass = mass ? mass
+                : reinterpret_cast<float*>(ws_at(
+                      workspace, L.track_off + align_up((size_t)B * H * N * sizeof(float), 256)));
+  return from_cuda(launch_track(a, static_cast<cudaStream_t>(stream)));
 }
 
 fdllm_status fdllm_get_status(void* workspace, void* stream) {

@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(128) attn_simt(AttnArgs a) {
     }
     T* o = static_cast<T*>(a.out) + ((size_t)b * rows + r) * a.H * dh + h * dh + d;
     Store<T>::st(o, num / den);
+    if (d == 0 && a.lse) a.lse[((size_t)b * rows + r) * a.H + h] = M + log2f(den);
   }
 }
 

@@ -58,6 +58,7 @@ struct AttnTcParams {
   const __nv_bfloat16* k_cache;  // [B, H, N, DH], for the L2 prefetch
   const __nv_bfloat16* v_cache;
   __nv_bfloat16* out;
+  float* lse;          // [B, rows, H] log2 softmax denominators, or null
   int* status;
   int cs;              // cluster size in cluster mode, 0 in stream-K mode
   float* partials;     // [grid][2][NQ*DH + 2*NQ]
@@ -663,6 +664,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               if (r < p.rows) {
                 const float lt = wred[cq] + wred[NQ + cq] + wred[2 * NQ + cq] + wred[3 * NQ + cq];
                 p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + kl] = __float2bfloat16_rn(o[c] / lt);
+                if (kl == 0 && p.lse) p.lse[((size_t)b * p.rows + r) * p.H + h] = alpha[cq] + log2f(lt);
               }
             }
           }
@@ -742,9 +744,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int r = qc * NQ + c4 + e;
-              if (r < p.rows)
+              if (r < p.rows) {
                 p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + row] =
                     __float2bfloat16_rn(Lsum[e] > 0.f ? acc[e] / Lsum[e] : 0.f);
+                if (row == 0 && p.lse) p.lse[((size_t)b * p.rows + r) * p.H + h] = M[e] + log2f(Lsum[e]);
+              }
             }
           }
           // no CTA leaves while another may still read its shared memory
@@ -818,6 +822,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
               }
             }
+            if (st < NQ && p.lse && qc * NQ + st < p.rows)
+              p.lse[((size_t)b * p.rows + qc * NQ + st) * p.H + h] = M + log2f(Lsum);
             constexpr int kJ = NQ == 64 ? 2 : 4;  // contributors per batch of O loads
             float acc[NQH];
 #pragma unroll
@@ -1071,6 +1077,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   prm.k_cache = static_cast<const __nv_bfloat16*>(a.k_cache);
   prm.v_cache = static_cast<const __nv_bfloat16*>(a.v_cache);
   prm.out = static_cast<__nv_bfloat16*>(a.out);
+  prm.lse = a.lse;
   prm.status = a.status;
   prm.partials = static_cast<float*>(a.ws);
   prm.item_cnt = reinterpret_cast<unsigned*>(static_cast<char*>(a.ws) + q.partial_bytes);

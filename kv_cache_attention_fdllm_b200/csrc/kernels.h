@@ -71,6 +71,8 @@ struct AttnArgs {
   const int8_t* view;      // verify only
   const int32_t* rank;     // verify only
   void* out;               // [B, rows, H*dh]
+  float* lse;              // [B, rows, H]: log2 of the softmax denominator of the
+                           // scaled scores s * log2(e) / sqrt(dh); may be null
   int* status;
   void* ws;
   size_t ws_bytes;
@@ -79,6 +81,24 @@ struct AttnArgs {
 size_t attn_workspace_bytes(int B, int N, int H, int dh, int rows_per_seq, int S_max, int verify,
                             int dtype, int num_sms);
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream);
+
+// ----------------------------------------------------------------- tracked-set selection
+constexpr int kMaxBetaT = FDLLM_MAX_BETA_T;
+
+struct TrackArgs {
+  int B, N, H, dh, nq, dtype, beta_t;
+  const void* q;            // [B, nq, H, dh], staged by the step
+  const float* lse;         // [B, nq, H], left by the step's attention
+  const int8_t* q_masked;   // [B, nq]: 1 = masked-query row
+  const int8_t* candidate;  // [B, N]: 1 = decoded slot
+  const void* k_cache;      // [B, H, N, dh]
+  int32_t* track;           // [B, beta_t]
+  float* mass;              // [B, N]
+  float* mass_h;            // [B, H, N] scratch
+};
+
+size_t track_workspace_bytes(int B, int N, int H);
+cudaError_t launch_track(const TrackArgs& a, cudaStream_t stream);
 
 // ----------------------------------------------------------------- kernel families
 size_t proj_simt_workspace_bytes(int M, int H, int dh);
