@@ -37,6 +37,7 @@ import workloads as W  # noqa: E402
 
 L2_FLUSH_BYTES = 512 << 20
 DEFAULT_WORKLOAD = "single_bf16"
+SWEEP_BATCHES = (1, 2, 4, 8, 16, 32, 64)
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -170,11 +171,12 @@ def traffic_for(kernel_key):
 
 # ------------------------------------------------------------------ our arm
 
-def run_ours(args, world, rank, local):
+def run_ours(args, world, rank, local, cfg=None, name=None, with_e2e=True):
     import kv_cache_attention_fdllm_b200 as F
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    cfg = W.CONFIGS[args.workload]
+    name = name or args.workload
+    cfg = cfg or W.CONFIGS[args.workload]
     B = cfg["B"]
     seqs = F.rank_sequences(B, rank)  # each rank owns its own sequences
     rope_base = cfg["rope_base"]
@@ -274,7 +276,7 @@ def run_ours(args, world, rank, local):
 
     # ---------------- end to end through the public call with host buffers
     e2e = None
-    if not verify:
+    if not verify and with_e2e:
         pin = {k: v.pin_memory() for k, v in host.items() if k in ("x", "q_idx")}
         out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         ws_e = F.alloc_workspace(ws.numel(), dev)
@@ -312,7 +314,7 @@ def run_ours(args, world, rank, local):
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
                 "algorithmic_bytes_per_launch": alg[dom],
-                "traffic": traffic_for(f"{args.workload}:{dom}"),
+                "traffic": traffic_for(f"{name}:{dom}"),
                 "ms_per_launch": stage_mean[dom]}
 
     res = {
@@ -322,7 +324,7 @@ def run_ours(args, world, rank, local):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": mean_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg["dtype"], "data": "synthetic",
-        "config": {"workload": workload_desc(args.workload, cfg),
+        "config": {"workload": workload_desc(name, cfg),
                    "l2": "flushed before every timed step (512 MB write)",
                    "parallelism": f"replicas x{world} (sequences sharded, no collective)"},
         "hbm_gbs_step": step_bytes / (mean_step / 1e3) / 1e9,
@@ -423,6 +425,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=[k for k in W.CONFIGS if k != "tiny_fp32"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep-batch", action="store_true",
+                    help="batch scaling study: the single-sequence shape (N = 512 prompt + 512 "
+                         "generated, |Q| = 32) at B = 1..64 per GPU, one JSON line per B")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -438,6 +443,19 @@ def main():
             "nccl", device_id=torch.device("cuda", local),
             timeout=__import__("datetime").timedelta(seconds=120))
     try:
+        if args.sweep_batch:
+            for B in SWEEP_BATCHES:
+                cfg = dict(W.CONFIGS["single_bf16"], B=B, seed=6)
+                r = run_ours(args, world, rank, local, cfg=cfg, name=f"sweep_B{B}", with_e2e=False)
+                if rank == 0:
+                    print(json.dumps({"sweep": "batch", "B_per_gpu": B, "n_gpus": world,
+                                      "value": r["value"], "unit": r["unit"],
+                                      "ms_per_step": r["ms_per_step"],
+                                      "hbm_gbs_step": r["hbm_gbs_step"],
+                                      "step_roofline_frac": r["step_roofline_frac"],
+                                      "stage_ms": r["stage_ms"], "clocks": r["clocks"],
+                                      "config": r["config"]}), flush=True)
+            return
         res = run_ours(args, world, rank, local)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             cfg = W.CONFIGS[args.workload]

@@ -509,7 +509,10 @@ ProjPlan plan(int M, int D, int H, int dh, int num_sms) {
   q.total_units = (long long)q.tiles * q.nks;
   q.grid = (int)(q.total_units < num_sms ? q.total_units : num_sms);
   q.smem_bytes = (size_t)q.nstage * stage + fixed;
-  q.partial_bytes = align_up((size_t)q.grid * 2 * q.BN * kBM * sizeof(float), 256);
+  // sized by min(256, M rounded up to 16) >= BN, not by BN itself: BN is not
+  // monotone in M, and a workspace sized for the most rows must serve fewer
+  const int bn_bound = (int)(((M + 15) / 16) * 16 < kMaxBN ? ((M + 15) / 16) * 16 : kMaxBN);
+  q.partial_bytes = align_up((size_t)q.grid * 2 * bn_bound * kBM * sizeof(float), 256);
   q.counter_bytes = align_up((size_t)q.tiles * sizeof(unsigned), 256);
   q.xq_bytes = align_up((size_t)M * D * 2, 256);
   return q;

@@ -63,6 +63,23 @@ def test_workspace_sizes(native):
 FAKE = ctypes.c_void_p(1 << 20)  # an aligned address that is never dereferenced
 
 
+def test_workspace_sizes_grow_with_rows(native):
+    """A workspace sized for the most rows serves every smaller row count (the
+    decode loop sizes one verify workspace for its largest pass)."""
+    lib = native.lib()
+    for dt in (0, 1):
+        prev = 0
+        for R in range(1, 513):
+            w = lib.fdllm_verify_step_workspace_bytes(8, 1024, 4096, 32, 128, R, 64, dt)
+            assert w >= prev, (dt, R, w, prev)
+            prev = w
+        prev = 0
+        for nq in range(1, 300):
+            w = lib.fdllm_fused_step_workspace_bytes(8, 1024, 4096, 32, 128, nq, dt)
+            assert w >= prev, (dt, nq, w, prev)
+            prev = w
+
+
 def test_bad_arguments_are_rejected_on_the_host(native):
     lib = native.lib()
     big = 1 << 40
