@@ -86,6 +86,12 @@ __device__ __forceinline__ int owner_of(long long u, long long total, int G) {
   return c;
 }
 
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* ptr) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -320,9 +326,24 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       tc::tc_fence_after();
 
       bool run = true;
+      bool own_in_tmem = true;  // this CTA's part of the tile is still (only) in TMEM
       int c_first = c, c_last = c;
       const long long tu0 = (long long)tile * p.nks;
       if (!whole) {
+        c_first = owner_of(tu0, p.total_units, G);
+        c_last = owner_of(tu0 + p.nks - 1, p.total_units, G);
+        // The other contributors count up after storing their parts.  When they
+        // all have, this CTA is the last one and merges its own part straight
+        // from TMEM: no store, fence or atomic of its own.
+        if (etid == 0) {
+          const unsigned done = ld_acquire(&p.tile_cnt[tile]);
+          *last_flag = (done == (unsigned)(c_last - c_first)) ? 2 : 0;
+          if (*last_flag == 2) p.tile_cnt[tile] = 0u;  // reset for the next call
+        }
+        tc::named_bar_sync(1, kEpiThreads);
+      }
+      if (!whole && *last_flag != 2) {
+        own_in_tmem = false;
         // partial tile: store it, free the accumulator, and see who is last
         const int slot = (j == 0) ? 0 : 1;
         float* dst = my_parts + (size_t)slot * BN * kBM;
@@ -337,8 +358,6 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&acc_empty[buf]);
         __threadfence();
-        c_first = owner_of(tu0, p.total_units, G);
-        c_last = owner_of(tu0 + p.nks - 1, p.total_units, G);
         tc::named_bar_sync(1, kEpiThreads);
         if (etid == 0) {
           const unsigned prev = atomicAdd(&p.tile_cnt[tile], 1u);
@@ -364,37 +383,31 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
 #pragma unroll
               for (int n = 0; n < kChunk / 2; ++n) staging[f_loc * kPitch + n_half + n] = v[n];
             }
-          } else {
-            // sum the partials of every contributor in k order; a thread adds
-            // 4 consecutive features of 4 tokens with 16-byte loads
-            constexpr int kTok = kChunk * (kBM / 4) / kEpiThreads;  // 4
-            constexpr int kStride = kEpiThreads / (kBM / 4);        // 8
-            float4 acc[kTok];
+          } else if (cc + n_half < BN) {
+            // sum the parts of every contributor in CTA (k) order, the thread's
+            // feature row over its 16 tokens: this CTA's part from TMEM when it
+            // was never stored, the others' from global memory
+            float v[kChunk / 2];
 #pragma unroll
-            for (int i = 0; i < kTok; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            const int f4 = (etid & 31) * 4;
-            const int nb = etid >> 5;  // tokens nb, nb + 8, ...
+            for (int n = 0; n < kChunk / 2; ++n) v[n] = 0.f;
             for (int cb = c_first; cb <= c_last; ++cb) {
-              // slot 0 when the tile is cb's first: unit_lo(cb) >= tu0
-              const int sl = (p.total_units * cb >= tu0 * (long long)G) ? 0 : 1;
-              const float* ps = p.partials + ((size_t)cb * 2 + sl) * BN * kBM;
+              float t[kChunk / 2];
+              if (cb == c && own_in_tmem) {
+                tc::tmem_ld16(t_acc + cc + n_half, t);
+                tc::tmem_wait_ld();
+              } else {
+                // slot 0 when the tile is cb's first: unit_lo(cb) >= tu0
+                const int sl = (p.total_units * cb >= tu0 * (long long)G) ? 0 : 1;
+                const float* ps = p.partials + ((size_t)cb * 2 + sl) * BN * kBM +
+                                  (size_t)(cc + n_half) * kBM + f_loc;
 #pragma unroll
-              for (int i = 0; i < kTok; ++i) {
-                const int n = cc + nb + kStride * i;
-                if (n < BN) {
-                  const float4 t = __ldcg(reinterpret_cast<const float4*>(ps + (size_t)n * kBM + f4));
-                  acc[i].x += t.x; acc[i].y += t.y; acc[i].z += t.z; acc[i].w += t.w;
-                }
+                for (int n = 0; n < kChunk / 2; ++n) t[n] = __ldcg(ps + (size_t)n * kBM);
               }
+#pragma unroll
+              for (int n = 0; n < kChunk / 2; ++n) v[n] += t[n];
             }
 #pragma unroll
-            for (int i = 0; i < kTok; ++i) {
-              const int n = nb + kStride * i;
-              staging[(f4 + 0) * kPitch + n] = acc[i].x;
-              staging[(f4 + 1) * kPitch + n] = acc[i].y;
-              staging[(f4 + 2) * kPitch + n] = acc[i].z;
-              staging[(f4 + 3) * kPitch + n] = acc[i].w;
-            }
+            for (int n = 0; n < kChunk / 2; ++n) staging[f_loc * kPitch + n_half + n] = v[n];
           }
           tc::named_bar_sync(1, kEpiThreads);
           // 32 tokens x 16 groups of 8 features; a warp covers 32 tokens of one group
@@ -455,7 +468,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           tc::named_bar_sync(1, kEpiThreads);
         }
       }
-      if (whole) {
+      if (whole || own_in_tmem) {
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&acc_empty[buf]);
