@@ -31,7 +31,13 @@
 //
 //   warp 0      TMA producer: Q chunk per item, K and V tiles (128 x 64 boxes)
 //   warp 1      TMEM allocation; lane 0 issues QK (ahead by one tile) and PV
-//   warps 2-5   softmax over S^T, P, accumulator rescale, epilogue
+//   warps 2..   softmax over S^T, P, accumulator rescale, epilogue: NQ/kCols
+//               groups of 4 warps (8 warps at NQ = 32 and 64, 4 at NQ = 16)
+//
+// Launched as a programmatic dependent: the prologue and an L2 prefetch of
+// the first cache tiles run before the grid-dependency wait; every thread
+// waits before it reads anything an earlier kernel wrote.  The kernel leaves
+// each row's log2 softmax normaliser (per head) for the tracked-set selection.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
