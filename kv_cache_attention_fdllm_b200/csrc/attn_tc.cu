@@ -38,6 +38,8 @@
 // the first cache tiles run before the grid-dependency wait; every thread
 // waits before it reads anything an earlier kernel wrote.  The kernel leaves
 // each row's log2 softmax normaliser (per head) for the tracked-set selection.
+#include <limits.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -218,6 +220,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   int* last_flag = abort_flag + 1;
   int* n_draft_s = last_flag + 1;
   int* n_side_s = n_draft_s + 1;
+  int* d_lo_s = n_side_s + 1;  // smallest and largest draft position of the segment
+  int* d_hi_s = d_lo_s + 1;
   float* m_run = reinterpret_cast<float*>(misc + 512);      // [NQ]
   float* alpha = m_run + 128;                               // [NQ]
   float* wred = alpha + 128;                                // [4][NQ]
@@ -450,7 +454,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const float scale = p.qk_scale;
     float l[NQH], mrun[NQH];
     int seg = -1;
-    int n_draft = 0, n_side = 0;
+    int n_draft = 0, n_side = 0, d_lo = INT_MAX, d_hi = INT_MIN;
     int pv_waited = -1;  // index of the last PV this thread waited for
     int seg_t0 = 0;      // tile index at which the current segment started
     UnitCursor cs;
@@ -474,24 +478,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           if (warp == 2 || warp == 3) {
             // ballot compaction of draft rows (warp 2) and mask rows (warp 3)
             const int want = warp == 2 ? 1 : 2;
-            int base = 0;
+            int base = 0, lo = INT_MAX, hi = INT_MIN;
             for (int r = lane; r - lane < p.rows; r += 32) {
               const int vw = r < p.rows ? (int)p.view[r0 + r] : -1;
               const unsigned bal = __ballot_sync(0xffffffffu, vw == want);
               const int at = base + __popc(bal & ((1u << lane) - 1u));
               if (vw == want && at < kMaxRows) {
                 if (want == 1) {
-                  draft_pos[at] = p.pos[r0 + r];
+                  const int ps = p.pos[r0 + r];
+                  draft_pos[at] = ps;
                   draft_rank[at] = p.rank[r0 + r];
+                  lo = min(lo, ps);
+                  hi = max(hi, ps);
                 } else {
                   side_rank[at] = p.rank[r0 + r];
                 }
               }
               base += __popc(bal);
             }
+            lo = __reduce_min_sync(0xffffffffu, lo);
+            hi = __reduce_max_sync(0xffffffffu, hi);
             if (lane == 0) {
-              if (want == 1) *n_draft_s = min(base, kMaxRows);
-              else *n_side_s = min(min(base, p.S_max), kMaxRows);
+              if (want == 1) {
+                *n_draft_s = min(base, kMaxRows);
+                *d_lo_s = lo;
+                *d_hi_s = hi;
+              } else {
+                *n_side_s = min(min(base, p.S_max), kMaxRows);
+              }
             }
           }
         }
@@ -504,6 +518,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (VERIFY) {
           n_draft = *n_draft_s;
           n_side = *n_side_s;
+          d_lo = *d_lo_s;
+          d_hi = *d_hi_s;
         }
       }
 
@@ -535,9 +551,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (!visible_side(cm & 3, cm >> 2, srank, p.causal)) s[c] = -INFINITY;
           }
         } else {
+          // only tiles that reach the draft positions' range need the lookup
           int kdr = -1;
-          for (int d = 0; d < n_draft; ++d)
-            if (draft_pos[d] == key) kdr = draft_rank[d];
+          const int tk0 = t * kKT;
+          if (tk0 <= d_hi && tk0 + kKT > d_lo)
+            for (int d = 0; d < n_draft; ++d)
+              if (draft_pos[d] == key) kdr = draft_rank[d];
           if (kdr >= 0) {
 #pragma unroll
             for (int c = 0; c < NQH; ++c) {
