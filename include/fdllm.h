@@ -104,7 +104,9 @@ size_t fdllm_accept_workspace_bytes(int B, int R, int V);
  *   ([review] "Flash-Verify": Q_t = T_t u M_t^{beta_m}); slots within [0, N),
  *   distinct within a row, any order.  An index outside [0, N) sets
  *   FDLLM_ERR_BAD_INDEX in the status word and that row is skipped (nothing is
- *   written for it).  Duplicates are undefined.
+ *   written for it).  A repeated index also sets FDLLM_ERR_BAD_INDEX (both rows
+ *   write the same slot; which write lands is undefined); bf16 only, the fp32
+ *   path does not check.
  *   k_cache / v_cache are read and written in place: only the slots in Q
  *   change.  x must not alias any buffer the call writes.
  *   out [B, nq, H*dh]: row i is the attention output of query q_idx[b, i]. */

@@ -98,16 +98,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 }
 
 // One CTA per projection row m of the fused step: xq[m] = x[b, q_idx[m]] (zeros
-// when the index is out of range).
+// when the index is out of range); a repeated index sets FDLLM_ERR_BAD_INDEX.
 __global__ void __launch_bounds__(128) proj_prep_kernel(const __nv_bfloat16* __restrict__ x,
                                                         const int32_t* __restrict__ idx, int N,
                                                         int D, int rows_per_seq,
-                                                        __nv_bfloat16* __restrict__ xq) {
+                                                        __nv_bfloat16* __restrict__ xq,
+                                                        int* __restrict__ status) {
   tc::griddep_launch_dependents();
   const int m = blockIdx.x;
   const int ps = idx[m];
   const bool ok = ps >= 0 && ps < N;
   const int b = m / rows_per_seq;
+  // Q is a set: an index that repeats an earlier row of the sequence is
+  // reported (both rows would write the same cache slot)
+  for (int r = b * rows_per_seq + threadIdx.x; r < m; r += blockDim.x)
+    if (idx[r] == ps) set_status(status, FDLLM_ERR_BAD_INDEX);
   const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)b * N + (ok ? ps : 0)) * D);
   uint4* dst = reinterpret_cast<uint4*>(xq + (size_t)m * D);
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
@@ -587,7 +592,7 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream) {
   if (!a.verify) {
     // the fused step gathers x[Q] into a packed operand; verify rows arrive packed
     proj_prep_kernel<<<M, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.x), a.idx, a.N,
-                                            a.D, a.rows_per_seq, xq);
+                                            a.D, a.rows_per_seq, xq, a.status);
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -122,6 +122,46 @@ def test_out_of_range_index_sets_status_and_skips_row(F):
     assert F.fdllm_get_status(ws) == F.OK  # read-and-clear
 
 
+def test_repeated_index_sets_status(F):
+    """Q is a set; a repeated slot is reported through the status word."""
+    inp = W.random_fused(2, 100, 128, 2, 64, q_idx=np.array([[3, 9, 3], [5, 6, 7]]), seed=11)
+    dev = W.to_device(inp)
+    out, ws, st = run_fused_gpu(F, dev, 10000.0)
+    assert st == F.ERR_BAD_INDEX
+    inp = W.random_fused(2, 100, 128, 2, 64, q_idx=np.array([[3, 9, 4], [5, 6, 7]]), seed=11)
+    out, ws, st = run_fused_gpu(F, W.to_device(inp), 10000.0)
+    assert st == F.OK
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_guard_sequences_around_the_buffers_stay_intact(F, dtype):
+    """The caches and the output sit inside larger allocations whose extra
+    sequences before and after are filled with a NaN pattern: the call must
+    leave them bit-identical (no write past its own buffers)."""
+    B, N, D, H, dh, nq = 2, 300, 128, 2, 64, 9
+    inp = W.random_fused(B, N, D, H, dh, nq=nq, dtype=dtype, seed=12)
+    dev = W.to_device(inp)
+    t = dev["k_cache"].dtype
+    guard = float("nan")
+    kb = torch.full((B + 2, H, N, dh), guard, dtype=t, device="cuda")
+    vb = torch.full((B + 2, H, N, dh), guard, dtype=t, device="cuda")
+    ob = torch.full((B + 2, nq, H * dh), guard, dtype=t, device="cuda")
+    kb[1:B + 1].copy_(dev["k_cache"])
+    vb[1:B + 1].copy_(dev["v_cache"])
+    before = [kb.clone(), vb.clone(), ob.clone()]
+    k, v, o = kb[1:B + 1], vb[1:B + 1], ob[1:B + 1]
+    assert k.is_contiguous() and o.is_contiguous()
+    ws = F.alloc_workspace(F.fdllm_fused_step_workspace_bytes(B, N, D, H, dh, nq, t), "cuda")
+    F.fdllm_fused_step(dev["x"], dev["q_idx"], dev["w_qkv"], k, v, o, ws)
+    assert F.fdllm_get_status(ws) == F.OK
+    for now, was in zip((kb, vb, ob), before):
+        for g in (0, B + 1):
+            a = now[g].contiguous().view(torch.int16 if t == torch.bfloat16 else torch.int32)
+            b = was[g].contiguous().view(torch.int16 if t == torch.bfloat16 else torch.int32)
+            assert torch.equal(a, b), "a guard sequence changed"
+    assert not torch.isnan(o).any()
+
+
 def test_empty_batch_is_a_no_op(F):
     x = torch.zeros((0, 10, 64), dtype=torch.bfloat16, device="cuda")
     q = torch.zeros((0, 2), dtype=torch.int32, device="cuda")
