@@ -932,6 +932,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 struct AttnPlan {
   int NQ, n_qc, nct, nst, tpi, nk, nv, grid;  // stream-K: rings, grid
   int cs, nk_cl, nv_cl;                        // cluster size wanted (0: stream-K), its rings
+  bool whole_items;                            // many items: one CTA per item, no merges
   long long items, total_units;
   size_t smem_bytes, smem_cl, partial_bytes, counter_bytes;
 };
@@ -977,6 +978,19 @@ AttnPlan plan(int B, int N, int H, int dh, int rows, int S_max, int verify, int 
   };
   q.smem_bytes = rings(2, q.nk, q.nv);
   q.smem_cl = rings(1, q.nk_cl, q.nv_cl);
+  // Many items in at most two waves: one CTA per whole item avoids the item
+  // boundaries inside a CTA's range - each costs the softmax warps an epilogue
+  // and a new item's setup while the next tile waits, about 6 tiles of time -
+  // and every merge.  Taken when its wave-quantised makespan is no longer than
+  // stream-K's plus two such boundaries.  With more waves every CTA's cold
+  // start (about 5 us) adds up, and persistent stream-K, which pipelines its
+  // loads across item boundaries, wins (measured: 2048 items, 649 -> 705 us).
+  q.whole_items = false;
+  if (q.cs == 0 && q.items > num_sms) {
+    const long long waves = (q.items + num_sms - 1) / num_sms;
+    const double sk_tiles = (double)q.total_units / num_sms + 2 * 6.0;
+    q.whole_items = waves <= 2 && (double)(waves * q.tpi) <= sk_tiles;
+  }
   q.partial_bytes = align_up((size_t)q.grid * 2 * ((size_t)q.NQ * dh + 2 * q.NQ) * sizeof(float), 256);
   q.counter_bytes = align_up((size_t)q.items * sizeof(unsigned), 256);
   return q;
@@ -1036,6 +1050,14 @@ cudaError_t launch_t(const AttnArgs& a, const AttnPlan& q, AttnTcParams prm, con
     cfg.gridDim = dim3((unsigned)(q.items * cs));
     cfg.dynamicSmemBytes = q.smem_cl;
     prm.cs = cs;
+    prm.nk = q.nk_cl;
+    prm.nv = q.nv_cl;
+    prm.nqbuf = 1;
+  } else if (q.whole_items) {
+    // grid = items: the unit split gives every CTA exactly one whole item
+    cfg.gridDim = dim3((unsigned)q.items);
+    cfg.dynamicSmemBytes = q.smem_cl;
+    prm.cs = 0;
     prm.nk = q.nk_cl;
     prm.nv = q.nv_cl;
     prm.nqbuf = 1;
