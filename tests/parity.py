@@ -7,8 +7,8 @@ import torch
 
 import oracle as O
 
-# Tolerances (stated by the task's matching rule): fp32 configurations max-abs
-# 1e-4; bf16 configurations max-abs relative to max|ref| 2e-2.
+# Tolerances of the matching rule: fp32 configurations max-abs 1e-4; bf16
+# configurations max-abs relative to max|ref| 2e-2.
 TOL_F32_ABS = 1e-4
 TOL_BF16_REL = 2e-2
 # conf is fp32 on the GPU, fp64 in the oracle; the sum over V terms carries
