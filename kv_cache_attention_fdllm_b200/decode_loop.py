@@ -22,9 +22,8 @@ Policies the pages leave to the caller (stated here, used below):
   * the exploratory set S of a step has the same size in every sequence (the
     smallest count over the batch), in decoding order (confidence descending);
   * the tracked set is chosen from the middle layer's attention.  The slots
-    resolved in the step join the ranking (the page includes them before
-    ranking): the middle layer ranks the decoded slots and the step's masked
-    positions, and T becomes the first beta_t of that ranking that are decoded
+    resolved in the step take part in the ranking, as on the page: the middle
+    layer ranks the decoded slots and the step's masked positions, and T becomes the first beta_t of that ranking that are decoded
     once the step has committed its rows.
 """
 from __future__ import annotations

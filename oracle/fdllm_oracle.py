@@ -27,7 +27,8 @@ What is computed (each function states its passage):
                    and the worked example).
   * attention_mass, track_select - the tracked set of the next step ([review],
                    "How It Works", Step 1: Cache selection): the decoded slots
-                   most attended by the masked queries.
+                   that receive the largest share of the masked queries'
+                   attention.
 
 Everything is computed in float64 from the exactly upcast stored inputs.  The
 k,v written into the cache are rounded once to the storage dtype, and the
@@ -352,8 +353,9 @@ def track_select(a, candidate, beta_t):
     selection): the beta_t candidate slots with the largest attention mass.
 
     candidate[b, j] != 0 marks a decoded slot.  The positions decoded in this
-    step are candidates like the earlier ones (the page includes the newly
-    resolved positions before ranking and keeps |T| at beta_t).  Order: mass
+    step are candidates like the earlier ones (on the page, the positions
+    resolved in the step take part in the ranking and T keeps beta_t
+    entries).  Order: mass
     descending, equal mass to the lower slot.  With fewer candidates than
     beta_t the tail is -1.  Returns int64 [B, beta_t]."""
     B, N = a.shape
