@@ -108,3 +108,22 @@ def test_bad_arguments_are_rejected_on_the_host(native):
              None) == 1                                       # V = 0
     assert a(1, 3, 3, FAKE, FAKE, None, None, 0.9, 0.8, FAKE, FAKE, FAKE, FAKE, FAKE, 0,
              None) == 6                                       # workspace too small
+
+
+def test_track_select_rejects_bad_arguments_on_the_host(native):
+    lib = native.lib()
+    big = 1 << 40
+    t = lib.fdllm_track_select
+    args = lambda beta=80, dh=128, ws=FAKE, wsb=big, qm=FAKE, mass=None: (
+        1, 1024, 32, dh, 32, 1, qm, FAKE, FAKE, beta, FAKE, mass, ws, wsb, None)
+    assert t(*args(beta=0)) == 2                     # beta_t out of range
+    assert t(*args(beta=1025)) == 2
+    assert t(*args(dh=96)) == 2                      # unsupported head size
+    assert t(*args(ws=None)) == 6                    # no workspace
+    assert t(*args(wsb=10)) == 6                     # smaller than the fused step's
+    assert t(*args(qm=None)) == 1                    # null tensor
+    assert t(*args(mass=ctypes.c_void_p((1 << 20) + 4))) == 1   # misaligned optional output
+    # the workspace a fused step of the same shape gets is large enough
+    need = lib.fdllm_fused_step_workspace_bytes(1, 1024, 4096, 32, 128, 32, 1)
+    assert need > 0
+    assert t(0, 1024, 32, 128, 32, 1, None, None, None, 80, None, None, FAKE, need, None) == 0
