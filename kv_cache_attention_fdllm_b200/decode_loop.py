@@ -85,6 +85,40 @@ def algorithmic_bytes_per_layer(cfg: LoopConfig, nq: int) -> dict:
     return {"fused": fused, "full_recompute": full}
 
 
+def query_set(decoded, T, beta_m):
+    """Q of the next step: the tracked set T, then the front beta_m masked
+    positions in position order.  When fewer masks remain, decoded slots that
+    are not in T fill the rest, flagged as non-masked rows.
+
+    decoded bool [B, N], T int32 [B, beta_t].  Returns (q_idx int32 [B, beta_t +
+    beta_m], q_masked int8 [B, beta_t + beta_m], front int64 [B, beta_m])."""
+    B, N = decoded.shape
+    dev = decoded.device
+    ar = torch.arange(N, device=dev)
+    masks_left = (~decoded).sum(dim=1)
+    key = torch.where(decoded, N + ar, ar)               # masks first, in position order
+    front = torch.argsort(key.float(), dim=1)[:, :beta_m]
+    m_cnt = torch.clamp(masks_left, max=beta_m)
+    is_T = torch.zeros((B, N), dtype=torch.bool, device=dev)
+    is_T.scatter_(1, T.long(), True)
+    fill = torch.argsort((is_T | ~decoded).float() * 2 + (ar.float() / N), dim=1)  # decoded, non-T
+    slot_j = torch.arange(beta_m, device=dev).unsqueeze(0)
+    front = torch.where(slot_j < m_cnt.unsqueeze(1), front, fill[:, :beta_m])
+    q_idx = torch.cat([T.int(), front.int()], dim=1).contiguous()
+    q_masked = torch.cat([torch.zeros((B, T.shape[1]), dtype=torch.int8, device=dev),
+                          (slot_j < m_cnt.unsqueeze(1)).to(torch.int8)], dim=1).contiguous()
+    return q_idx, q_masked, front
+
+
+def next_tracked(ranked, decoded, beta_t):
+    """The next tracked set: the first beta_t slots of the ranking (-1 entries
+    skipped) that are decoded once the step has committed its rows, in rank
+    order.  ranked int32 [B, K], decoded bool [B, N]."""
+    ok = (ranked >= 0) & torch.gather(decoded, 1, ranked.clamp(min=0).long())
+    first = torch.argsort((~ok).to(torch.int8), dim=1, stable=True)[:, :beta_t]
+    return torch.gather(ranked, 1, first).contiguous()
+
+
 def run(cfg: LoopConfig, device="cuda") -> dict:
     dev = torch.device(device)
     gen = torch.Generator(device=dev)
@@ -115,7 +149,6 @@ def run(cfg: LoopConfig, device="cuda") -> dict:
     decoded[:, : cfg.n_prompt] = True
     T = torch.arange(cfg.n_prompt - cfg.beta_t, cfg.n_prompt, device=dev, dtype=torch.int32)
     T = T.unsqueeze(0).expand(B, -1).contiguous()
-    ar = torch.arange(N, device=dev)
 
     steps, committed_total = 0, 0
     per_step_ms, per_step_commit = [], []
@@ -127,20 +160,7 @@ def run(cfg: LoopConfig, device="cuda") -> dict:
             break  # a finished sequence rides along with an all-decoded Q until then
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ev0.record()
-        # Q = T + the front beta_m masks (fewer masks left: more decoded slots
-        # fill Q, flagged as non-masked rows)
-        key = torch.where(decoded, N + ar, ar)            # masks first, in position order
-        order = torch.argsort(key.float(), dim=1)
-        m_cnt = torch.clamp(masks_left, max=cfg.beta_m)
-        front = order[:, : cfg.beta_m]
-        is_T = torch.zeros((B, N), dtype=torch.bool, device=dev)
-        is_T.scatter_(1, T.long(), True)
-        fill = torch.argsort((is_T | ~decoded).float() * 2 + (ar.float() / N), dim=1)  # decoded, non-T
-        slot_j = torch.arange(cfg.beta_m, device=dev).unsqueeze(0)
-        front = torch.where(slot_j < m_cnt.unsqueeze(1), front, fill[:, : cfg.beta_m])
-        q_idx = torch.cat([T, front.int()], dim=1).contiguous()
-        q_masked = torch.cat([torch.zeros((B, cfg.beta_t), dtype=torch.int8, device=dev),
-                              (slot_j < m_cnt.unsqueeze(1)).to(torch.int8)], dim=1).contiguous()
+        q_idx, q_masked, front = query_set(decoded, T, cfg.beta_m)
 
         # draft pass over the layers; the tracked set comes from the middle layer
         x = x0.clone()
@@ -215,10 +235,7 @@ def run(cfg: LoopConfig, device="cuda") -> dict:
             newly[none, bpos[none]] = True
         newly &= ~decoded
         decoded |= newly
-        # T: the first beta_t ranked slots that are decoded now, in rank order
-        ok = (track >= 0) & torch.gather(decoded, 1, track.clamp(min=0).long())
-        first = torch.argsort((~ok).to(torch.int8), dim=1, stable=True)[:, : cfg.beta_t]
-        T = torch.gather(track, 1, first).contiguous()
+        T = next_tracked(track, decoded, cfg.beta_t)
         ev1.record()
         torch.cuda.synchronize()
         for w in (ws, ws_v, ws_a):
