@@ -333,6 +333,21 @@ def test_accept_prefix_stops_at_first_failure():
         assert [(int(x) & O.FLAG_PASS) > 0 for x in f[0]] == [True, False, True]
 
 
+def test_accept_thresholds_are_inclusive():
+    """Two equal logits give a confidence of exactly 1/2.  At eps = gamma = 1/2
+    the draft row is committed and the mask-view row passes (the worked
+    example's margins leave the boundary open; the reading is c >= eps and
+    c~ >= gamma).  One ulp above 1/2, neither."""
+    l = np.zeros((1, 2, 2))
+    kind, ref, rank = np.array([[1, 2]]), np.array([[-1, 0]]), np.array([[-1, 0]])
+    _, c, f, n = O.accept(l, kind, ref, rank, 0.5, 0.5)
+    assert c[0].tolist() == [0.5, 0.5]
+    assert f[0, 0] & O.FLAG_COMMIT and f[0, 1] & O.FLAG_PASS and n[0] == 1
+    up = float(np.nextafter(0.5, 1.0))
+    _, _, f, n = O.accept(l, kind, ref, rank, up, up)
+    assert not f[0, 0] & O.FLAG_COMMIT and not f[0, 1] & O.FLAG_PASS and n[0] == 0
+
+
 def test_accept_ties_uniform_and_tv_bound():
     g = np.random.default_rng(9)
     l = np.zeros((1, 2, 50))
