@@ -3,7 +3,8 @@
 Each function has the name of the C entry point it calls (include/fdllm.h),
 takes torch CUDA tensors, checks their dtype, shape, device and contiguity,
 passes raw pointers and the current CUDA stream, and raises FdllmError on a
-non-OK status.  Every step of the computation runs in the CUDA library.
+non-OK status.  The library launches on the current CUDA device, so the tensors
+and the stream must be on it (a ValueError otherwise).  Every step of the computation runs in the CUDA library.
 """
 from __future__ import annotations
 
@@ -34,8 +35,18 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
 
 
-def _stream(stream):
-    s = torch.cuda.current_stream() if stream is None else stream
+def _stream(stream, device):
+    """The stream handle to launch on.  The library launches on the current CUDA
+    device, so the tensors (on `device`) and the stream must both be on it."""
+    if device.type != "cuda":
+        raise ValueError(f"the tensors are on {device}, not on a CUDA device")
+    cur = torch.cuda.current_device()
+    if device.index != cur:
+        raise ValueError(f"the tensors are on {device}, but the current CUDA device is "
+                         f"cuda:{cur} (use torch.cuda.set_device)")
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    if s.device != device:
+        raise ValueError(f"the stream is on {s.device}, the tensors on {device}")
     return ctypes.c_void_p(s.cuda_stream)
 
 
@@ -108,7 +119,7 @@ def fdllm_fused_step(x, q_idx, w_qkv, k_cache, v_cache, out, workspace, rope_bas
     _need(workspace, "workspace", torch.uint8, None, x.device)
     st = lib().fdllm_fused_step(B, N, D, H, dh, nq, _dtype_code(x), _p(x), _p(q_idx), _p(w_qkv),
                                 float(rope_base), _p(k_cache), _p(v_cache), _p(out),
-                                _p(workspace), workspace.numel(), _stream(stream))
+                                _p(workspace), workspace.numel(), _stream(stream, x.device))
     _check(st, "fdllm_fused_step")
     return out
 
@@ -121,7 +132,7 @@ def fdllm_qkv_rope_scatter(x, q_idx, w_qkv, k_cache, v_cache, q_out, workspace,
     st = lib().fdllm_qkv_rope_scatter(B, N, D, H, dh, nq, _dtype_code(x), _p(x), _p(q_idx),
                                       _p(w_qkv), float(rope_base), _p(k_cache), _p(v_cache),
                                       _p(q_out), _p(workspace), workspace.numel(),
-                                      _stream(stream))
+                                      _stream(stream, x.device))
     _check(st, "fdllm_qkv_rope_scatter")
     return q_out
 
@@ -135,7 +146,7 @@ def fdllm_attend(q, k_cache, v_cache, out, workspace, stream=None):
     _need(out, "out", q.dtype, (B, nq, H * dh), q.device)
     _need(workspace, "workspace", torch.uint8, None, q.device)
     st = lib().fdllm_attend(B, N, H, dh, nq, _dtype_code(q), _p(q), _p(k_cache), _p(v_cache),
-                            _p(out), _p(workspace), workspace.numel(), _stream(stream))
+                            _p(out), _p(workspace), workspace.numel(), _stream(stream, q.device))
     _check(st, "fdllm_attend")
     return out
 
@@ -170,7 +181,7 @@ def fdllm_verify_step(x_rows, pos, view, rank, w_qkv, k_cache, v_cache, k_side, 
                                  _p(pos), _p(view), _p(rank), _p(w_qkv), float(rope_base),
                                  _p(k_cache), _p(v_cache), _p(k_side), _p(v_side), _p(out),
                                  int(bool(causal_cross)), _p(workspace), workspace.numel(),
-                                 _stream(stream))
+                                 _stream(stream, x_rows.device))
     _check(st, "fdllm_verify_step")
     return out
 
@@ -185,7 +196,7 @@ def fdllm_verify_qkv_rope_scatter(x_rows, pos, view, w_qkv, k_cache, v_cache, k_
                                              _p(x_rows), _p(pos), _p(view), _p(w_qkv),
                                              float(rope_base), _p(k_cache), _p(v_cache),
                                              _p(k_side), _p(v_side), _p(q_out), _p(workspace),
-                                             workspace.numel(), _stream(stream))
+                                             workspace.numel(), _stream(stream, x_rows.device))
     _check(st, "fdllm_verify_qkv_rope_scatter")
     return q_out
 
@@ -209,7 +220,7 @@ def fdllm_verify_attend(q, pos, view, rank, k_cache, v_cache, k_side, v_side, ou
     st = lib().fdllm_verify_attend(B, N, H, dh, R, S_max, _dtype_code(q), _p(q), _p(pos),
                                    _p(view), _p(rank), _p(k_cache), _p(v_cache), _p(k_side),
                                    _p(v_side), _p(out), int(bool(causal_cross)), _p(workspace),
-                                   workspace.numel(), _stream(stream))
+                                   workspace.numel(), _stream(stream, dev))
     _check(st, "fdllm_verify_attend")
     return out
 
@@ -237,7 +248,7 @@ def fdllm_track_select(q_masked, candidate, k_cache, track, workspace, mass=None
     _need(workspace, "workspace", torch.uint8, None, dev)
     st = lib().fdllm_track_select(B, N, H, dh, nq, _dtype_code(k_cache), _p(q_masked),
                                   _p(candidate), _p(k_cache), track.shape[1], _p(track), _p(mass),
-                                  _p(workspace), workspace.numel(), _stream(stream))
+                                  _p(workspace), workspace.numel(), _stream(stream, dev))
     _check(st, "fdllm_track_select")
     return track, mass
 
@@ -260,7 +271,7 @@ def fdllm_accept(logits, kind, ref_tok, rank, top1, conf, flags, n_accept, works
     _need(workspace, "workspace", torch.uint8, None, dev)
     st = lib().fdllm_accept(B, R, V, _p(logits), _p(kind), _p(ref_tok), _p(rank), float(eps),
                             float(gamma), _p(top1), _p(conf), _p(flags), _p(n_accept),
-                            _p(workspace), workspace.numel(), _stream(stream))
+                            _p(workspace), workspace.numel(), _stream(stream, dev))
     _check(st, "fdllm_accept")
     return top1, conf, flags, n_accept
 
@@ -284,11 +295,11 @@ def fdllm_accept_noalloc(logits, kind, ref_tok, rank, top1, conf, flags, n_accep
     _need(n_accept, "n_accept", torch.int32, (B,), dev)
     st = lib().fdllm_accept_noalloc(B, R, V, _p(logits), _p(kind), _p(ref_tok), _p(rank),
                                     float(eps), float(gamma), _p(top1), _p(conf), _p(flags),
-                                    _p(n_accept), _stream(stream))
+                                    _p(n_accept), _stream(stream, dev))
     _check(st, "fdllm_accept_noalloc")
     return top1, conf, flags, n_accept
 
 
 def fdllm_get_status(workspace, stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device status word."""
-    return int(lib().fdllm_get_status(_p(workspace), _stream(stream)))
+    return int(lib().fdllm_get_status(_p(workspace), _stream(stream, workspace.device)))

@@ -127,3 +127,27 @@ def test_track_select_rejects_bad_arguments_on_the_host(native):
     need = lib.fdllm_fused_step_workspace_bytes(1, 1024, 4096, 32, 128, 32, 1)
     assert need > 0
     assert t(0, 1024, 32, 128, 32, 1, None, None, None, 80, None, None, FAKE, need, None) == 0
+
+
+def test_binding_launches_only_on_the_tensors_device(native, monkeypatch):
+    """The library launches on the current CUDA device: the binding refuses
+    tensors on another device, and a stream on another device (faked devices:
+    no GPU is needed)."""
+    import torch
+    from kv_cache_attention_fdllm_b200 import api
+
+    class FakeStream:
+        def __init__(self, index, handle):
+            self.device = torch.device("cuda", index)
+            self.cuda_stream = handle
+
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 1)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: FakeStream(1, 0x1234))
+    assert api._stream(None, torch.device("cuda", 1)).value == 0x1234
+    assert api._stream(FakeStream(1, 0x99), torch.device("cuda", 1)).value == 0x99
+    with pytest.raises(ValueError, match="current CUDA device"):
+        api._stream(None, torch.device("cuda", 0))
+    with pytest.raises(ValueError, match="the stream is on"):
+        api._stream(FakeStream(0, 0x99), torch.device("cuda", 1))
+    with pytest.raises(ValueError, match="not on a CUDA device"):
+        api._stream(None, torch.device("cpu"))
