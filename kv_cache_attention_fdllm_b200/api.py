@@ -4,7 +4,8 @@ Each function has the name of the C entry point it calls (include/fdllm.h),
 takes torch CUDA tensors, checks their dtype, shape, device and contiguity,
 passes raw pointers and the current CUDA stream, and raises FdllmError on a
 non-OK status.  The library launches on the current CUDA device, so the tensors
-and the stream must be on it (a ValueError otherwise).  Every step of the computation runs in the CUDA library.
+and the stream must be on it (a ValueError otherwise).  Every step of the
+computation runs in the CUDA library.
 """
 from __future__ import annotations
 
