@@ -28,6 +28,8 @@
  *     stated otherwise; the library allocates no device memory and keeps no
  *     per-call state between calls.  `stream` is a cudaStream_t (NULL = legacy
  *     default stream).  Calls are asynchronous on `stream`.
+ *   - Kernels launch on the calling thread's current CUDA device; every pointer
+ *     and `stream` must belong to that device.
  *   - The return value reports host-side validation and launch errors only.
  *     Errors the GPU detects (an index out of range, a bounded wait that ran
  *     out) are recorded in a status word inside `workspace`; read them with
