@@ -28,6 +28,11 @@ MUTANTS = [
     ("bf16_via_float32", "round_bf16", "x = np.asarray(x, dtype=np.float64)",
      "x = np.asarray(x, dtype=np.float32).astype(np.float64)"),
     ("bf16_decode_shift", "bf16_bits_to_f64", "<< np.uint32(16)", "<< np.uint32(15)"),
+    ("bf16_tensor_read_as_integers", "to_f64",
+     "bf16_bits_to_f64(t.contiguous().view(dtype=_torch_int16()).numpy().view(np.uint16))",
+     "t.contiguous().view(dtype=_torch_int16()).numpy().astype(np.float64)"),
+    ("f32_not_rounded", "round_to",
+     "np.asarray(x, np.float64).astype(np.float32).astype(np.float64)", "np.asarray(x, np.float64)"),
     # RoPE
     ("rope_theta_exponent", "rope", "base ** (-2.0 * j / dh)", "base ** (-1.0 * j / dh)"),
     ("rope_theta_from_one", "rope", "j = np.arange(half, dtype=np.float64)",

@@ -55,6 +55,22 @@ def test_round_bf16_hand_cases():
     assert O.round_bf16(0.0) == 0.0
 
 
+def test_storage_decoding_and_f32_rounding_match_torch():
+    """to_f64 widens stored bf16 and fp32 tensors exactly as torch does, and
+    round_to(., "f32") is torch's float64 -> float32 conversion (the bf16
+    branch is checked above on float32 inputs: torch's float64 -> bfloat16
+    conversion goes through float32 and so rounds twice)."""
+    g = np.random.default_rng(10)
+    x = g.standard_normal(5000) * np.exp(g.uniform(-30, 30, 5000))
+    t64 = torch.from_numpy(x)
+    for dt in (torch.bfloat16, torch.float32):
+        t = t64.to(dt)
+        np.testing.assert_array_equal(O.to_f64(t), t.to(torch.float64).numpy())
+    np.testing.assert_array_equal(O.round_to(x, "f32"),
+                                  t64.to(torch.float32).to(torch.float64).numpy())
+    assert not np.array_equal(O.round_to(x, "f32"), x)
+
+
 # ---------------------------------------------------------------- RoPE
 
 def test_rope_hand_values():
