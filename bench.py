@@ -39,6 +39,7 @@ L2_FLUSH_BYTES = 512 << 20
 DEFAULT_WORKLOAD = "single_bf16"
 SWEEP_BATCHES = (1, 2, 4, 8, 16, 32, 64)
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal
 
 
 # ------------------------------------------------------------------ helpers
@@ -360,6 +361,7 @@ def run_ours(args, world, rank, local, cfg=None, name=None, with_e2e=True):
                    "parallelism": f"replicas x{world} (sequences sharded, no collective)"},
         "hbm_gbs_step": step_bytes / (mean_step / 1e3) / 1e9,
         "step_roofline_frac": step_bytes / (mean_step / 1e3) / 1e9 / peak,
+        "step_roofline_frac_nominal": step_bytes / (mean_step / 1e3) / 1e9 / NOMINAL_HBM_GBS,
         "stage_ms": stage_mean,
         "roofline": roofline,
         "e2e": e2e,
