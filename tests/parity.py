@@ -129,3 +129,33 @@ def check_accept(gpu, ref, kind, rank, eps, gamma):
             np.testing.assert_array_equal((f_g[b] & O.FLAG_ACCEPT) > 0, acc)
             assert n_g[b] == acc.sum()
     return int(amb.sum())
+
+
+def check_track(track, mass, ref, cand, beta_t, dt):
+    """A tracked-set selection from the GPU (track [B, beta_t], mass [B, N]) is
+    valid against the oracle's masses ref [B, N]: the masses match within the
+    tolerance; the first min(beta_t, candidates) entries are distinct
+    candidates in the GPU's own order (mass descending, equal mass to the lower
+    slot) and the rest are -1; and no candidate left out is heavier than a
+    chosen one beyond what the tolerance allows.  The GPU ranks by its own
+    masses, each within tol of the oracle's, so a chosen slot may be up to
+    2 tol lighter (in the oracle's masses) than one left out."""
+    scale = max(float(np.abs(ref).max()), 1e-30)
+    tol = (1e-4 if dt == "f32" else 2e-2) * scale
+    err = float(np.abs(mass - ref).max())
+    assert err <= tol, f"mass max error {err:.3e} > {tol:.3e}"
+    B, N = ref.shape
+    for b in range(B):
+        cands = np.nonzero(cand[b])[0]
+        k = min(beta_t, cands.size)
+        sel = track[b, :k]
+        assert (track[b, k:] == -1).all(), "padding past the candidates must be -1"
+        assert len(set(sel.tolist())) == k, "selected slots must be distinct"
+        assert all(cand[b, j] for j in sel), "selected slots must be candidates"
+        for t in range(k - 1):
+            a0, a1 = mass[b, sel[t]], mass[b, sel[t + 1]]
+            assert a0 > a1 or (a0 == a1 and sel[t] < sel[t + 1]), "order"
+        rest = np.setdiff1d(cands, sel)
+        if k and rest.size:
+            assert ref[b, sel].min() >= ref[b, rest].max() - 2 * tol, \
+                "a heavier candidate was left out"

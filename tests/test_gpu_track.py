@@ -12,7 +12,7 @@ import torch
 
 import oracle as O
 import workloads as W
-from parity import dtype_name
+from parity import check_track, dtype_name
 
 pytestmark = pytest.mark.gpu
 
@@ -64,29 +64,6 @@ def _oracle_mass(inp, masked, rope_base=10000.0):
                             H, dh, masked), dt
 
 
-def _check(track, mass, ref, cand, beta_t, dt):
-    scale = max(float(np.abs(ref).max()), 1e-30)
-    tol = (1e-4 if dt == "f32" else 2e-2) * scale
-    err = float(np.abs(mass - ref).max())
-    assert err <= tol, f"mass max error {err:.3e} > {tol:.3e}"
-    B, N = ref.shape
-    for b in range(B):
-        cands = np.nonzero(cand[b])[0]
-        k = min(beta_t, cands.size)
-        sel = track[b, :k]
-        assert (track[b, k:] == -1).all(), "padding past the candidates must be -1"
-        assert len(set(sel.tolist())) == k, "selected slots must be distinct"
-        assert all(cand[b, j] for j in sel), "selected slots must be candidates"
-        # the GPU's own order: mass descending, equal mass to the lower slot
-        for t in range(k - 1):
-            a0, a1 = mass[b, sel[t]], mass[b, sel[t + 1]]
-            assert a0 > a1 or (a0 == a1 and sel[t] < sel[t + 1]), "order"
-        # validity against the oracle: nothing left out is heavier than what was chosen
-        rest = np.setdiff1d(cands, sel)
-        if k and rest.size:
-            assert ref[b, sel].min() >= ref[b, rest].max() - tol, "a heavier candidate was left out"
-
-
 @pytest.mark.parametrize("cfg_name", ["tiny_fp32", "single_bf16"])
 def test_track_select_configs(F, cfg_name):
     cfg = W.CONFIGS[cfg_name]
@@ -97,7 +74,7 @@ def test_track_select_configs(F, cfg_name):
     beta_t = min(80, N)
     track, mass, _ = _run(F, inp, masked, cand, beta_t, cfg["rope_base"])
     ref, dt = _oracle_mass(inp, masked, cfg["rope_base"])
-    _check(track, mass, ref, cand, beta_t, dt)
+    check_track(track, mass, ref, cand, beta_t, dt)
 
 
 @pytest.mark.parametrize("shape", [
@@ -112,7 +89,7 @@ def test_track_select_shapes(F, shape, dtype):
     masked, cand = _masks(B, N, nq, inp["q_idx"].numpy(), seed=N)
     track, mass, _ = _run(F, inp, masked, cand, 16)
     ref, dt = _oracle_mass(inp, masked)
-    _check(track, mass, ref, cand, 16, dt)
+    check_track(track, mass, ref, cand, 16, dt)
 
 
 def test_track_select_exact_cases(F):

@@ -5,7 +5,9 @@ here gets the oracle's own result in place of the GPU's, which it must accept,
 and then that result with one planted mistake, made on the CPU, which it must
 reject: a value just past the tolerance, a non-finite value, a changed slot
 outside Q, a missed or misplaced scatter, a wrong token, confidence, flag or
-accepted count, a prefix that runs past a failure.
+accepted count, a prefix that runs past a failure, a tracked set that is out of
+order, repeats a slot, holds a non-candidate, pads wrongly or leaves out a
+heavier candidate.
 """
 import math
 
@@ -16,7 +18,7 @@ import torch
 import oracle as O
 import workloads as W
 from parity import (CONF_TOL, TOL_BF16_REL, TOL_F32_ABS, assert_close, check_accept,
-                    check_cache_update, oracle_fused)
+                    check_cache_update, check_track, oracle_fused)
 
 
 def test_assert_close_bounds():
@@ -141,3 +143,50 @@ def test_check_accept_near_a_threshold():
         check_accept(gpu([P | A, 0, P | A], 2, gamma - 1e-6), ref, kind, rank, eps, gamma)
     with pytest.raises(AssertionError):
         check_accept(gpu([P | A, 0, P], 2, gamma - 1e-6), ref, kind, rank, eps, gamma)
+
+
+def test_check_track_rejects_planted_mistakes():
+    B, N, D, H, dh, nq, beta_t = 2, 40, 64, 3, 64, 6, 8
+    inp = W.random_fused(B, N, D, H, dh, nq=nq, dtype="f32", seed=12)
+    K2, _, _ = oracle_fused(inp, H, dh, 10000.0, "f32")
+    g = np.random.default_rng(13)
+    masked = (g.random((B, nq)) < 0.5).astype(np.int8)
+    masked[:, 0] = 1
+    cand = (g.random((B, N)) < 0.6).astype(np.int8)
+    f = O.to_f64
+    ref = O.attention_mass(f(inp["x"]), inp["q_idx"].numpy(), f(inp["w_qkv"]), 10000.0, K2, H,
+                           dh, masked)
+    good = O.track_select(ref, cand, beta_t).astype(np.int32)
+    check_track(good, ref, ref, cand, beta_t, "f32")
+    tol = 1e-4 * np.abs(ref).max()
+
+    def planted(track=None, mass=None, cnd=cand):
+        with pytest.raises(AssertionError):
+            check_track(good if track is None else track, ref if mass is None else mass, ref,
+                        cnd, beta_t, "f32")
+
+    t = good.copy()
+    t[0, [1, 2]] = t[0, [2, 1]]                            # out of order
+    planted(track=t)
+    t = good.copy()
+    t[1, 3] = t[1, 2]                                      # a slot twice
+    planted(track=t)
+    t = good.copy()
+    t[0, -1] = int(np.nonzero(cand[0] == 0)[0][0])         # not a decoded slot
+    planted(track=t)
+    t = good.copy()
+    rest = np.setdiff1d(np.nonzero(cand[0])[0], good[0])
+    light = rest[np.argmin(ref[0, rest])]
+    assert ref[0, good[0, -1]] - ref[0, light] > 2 * tol   # a real gap, not a near tie
+    t[0, -1] = light                                       # still in descending order
+    planted(track=t)
+    m = ref.copy()
+    m[1, 7] += 1.5 * tol                                   # a mass past the tolerance
+    planted(mass=m)
+    few = np.zeros_like(cand)
+    few[:, [2, 9, 30]] = 1
+    short = O.track_select(ref, few, beta_t).astype(np.int32)
+    check_track(short, ref, ref, few, beta_t, "f32")
+    t = short.copy()
+    t[0, 3:] = 0                                           # padding must be -1
+    planted(track=t, cnd=few)
