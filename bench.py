@@ -92,6 +92,30 @@ def algorithmic_bytes(cfg):
     return out, rows
 
 
+def step_bytes_min(cfg):
+    """Bytes one whole step must move at least, by the method's definition: W_qkv,
+    the rows x[Q], the K, V of the cache slots the step does not write, the new
+    k, v (cache and side slots), the side slots read back, and the output (plus
+    the logits for a verify pass and its acceptance).  Unlike the per-kernel sum,
+    it counts neither the rotated q staged between the two kernels nor the
+    attention's re-read of the slots just written."""
+    e = 2 if cfg["dtype"] == "bf16" else 4
+    B, N, D, H, dh = cfg["B"], cfg["N"], cfg["D"], cfg["H"], cfg["dh"]
+    E = H * dh
+    if cfg["kind"] == "fused":
+        rows = cfg["n_track"] + cfg["beta_m"]
+        cache_rows, side_rows = rows, 0
+    else:
+        rows = cfg["n_tv"] + 2 * cfg["n_s"]
+        cache_rows, side_rows = cfg["n_tv"] + cfg["n_s"], cfg["n_s"]
+    M = B * rows
+    total = (3 * E * D * e + M * D * e + 2 * B * H * (N - cache_rows) * dh * e
+             + 2 * M * E * e + 2 * B * side_rows * E * e + M * E * e)
+    if cfg["kind"] == "verify":
+        total += M * cfg["vocab"] * 4
+    return total
+
+
 class ClockSampler:
     """Samples SM clock and clock-event reasons through NVML while running."""
     NAMES = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
@@ -337,7 +361,7 @@ def run_ours(args, world, rank, local, cfg=None, name=None, with_e2e=True):
     stage_mean = {k: sum(v) / len(v) for k, v in stage_ms.items()}
     dom = max(stage_mean, key=stage_mean.get)
     achieved = alg[dom] / (stage_mean[dom] / 1e3) / 1e9
-    step_bytes = sum(alg.values())
+    step_bytes = step_bytes_min(cfg)
     # what the stage call launches, timed together by the events around it
     kernels = {"proj": "proj_prep_kernel + proj_tc_kernel" if not verify else "proj_tc_kernel",
                "attn": "attn_tc_kernel", "accept": "accept_kernel"}
