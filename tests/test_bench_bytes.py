@@ -37,3 +37,17 @@ def test_kernel_bytes_bound_the_step_from_above(bench):
         cfg = W.CONFIGS[name]
         alg, _ = bench.algorithmic_bytes(cfg)
         assert sum(alg.values()) >= bench.step_bytes_min(cfg)
+
+
+def test_traffic_record_is_used_only_for_the_captured_source(bench):
+    """The ncu traffic of a kernel is reported only while its source still hashes to
+    the capture's; unknown keys give None."""
+    import hashlib
+    import json
+    import os
+    rec = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    for key, d in rec.items():
+        src = os.path.join(bench.ROOT, d["source"])
+        same = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] == d["source_sha256_16"]
+        assert bench.traffic_for(key) == (d["bytes_per_launch"] if same else None)
+    assert bench.traffic_for("no_such_workload:proj") is None
