@@ -36,7 +36,7 @@ import torch  # noqa: E402
 import workloads as W  # noqa: E402
 
 L2_FLUSH_BYTES = 512 << 20
-DEFAULT_WORKLOAD = "single_bf16"
+DEFAULT_WORKLOAD = "batch_bf16"
 SWEEP_BATCHES = (1, 2, 4, 8, 16, 32, 64)
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal
@@ -68,6 +68,29 @@ def workload_desc(name, cfg):
     return (f"{name}: verify pass + acceptance B={cfg['B']} N={cfg['N']} D={cfg['D']} "
             f"H={cfg['H']} dh={cfg['dh']} R={R} ({cfg['n_tv']} T_v + {cfg['n_s']} draft + "
             f"{cfg['n_s']} mask rows) V={cfg['vocab']} {cfg['dtype']}")
+
+
+def workload_with_overrides(args):
+    """The named workload, with --batch / --seq-len applied (name suffixed)."""
+    cfg = dict(W.CONFIGS[args.workload])
+    name = args.workload
+    if args.batch is not None:
+        cfg["B"] = args.batch
+        name += f"@B{args.batch}"
+    if args.seq_len is not None:
+        gen = cfg["N"] - cfg["n_prompt"]
+        if args.seq_len <= gen:
+            gen = args.seq_len // 2
+        cfg["N"], cfg["n_prompt"] = args.seq_len, args.seq_len - gen
+        name += f"@N{args.seq_len}"
+    return cfg, name
+
+
+def bench_config(name, cfg, world):
+    """The workload a line measures; the same dict in both arms of the bench."""
+    return {"workload": workload_desc(name, cfg),
+            "l2": "GPU arm: flushed before every timed step (512 MB write); host arm: n/a",
+            "parallelism": f"replicas x{world} (sequences sharded over ranks, no collective)"}
 
 
 def algorithmic_bytes(cfg):
@@ -325,13 +348,44 @@ def run_ours(args, world, rank, local, cfg=None, name=None, with_e2e=True):
     mean_step = F.max_over_ranks(sum(step_ms) / len(step_ms), dev)
     tokens_per_step = B * rows * world
 
-    # ---------------- end to end through the public call with host buffers
+    # ---------------- end to end through the public call with host buffers: every
+    # step copies its inputs from pinned host memory (the rows the step reads and
+    # their indices; for a verify pass also its metadata and the logits) and reads
+    # its results back; W and the caches are the resident state the step updates
     e2e = None
-    if not verify and with_e2e:
-        pin = {k: v.pin_memory() for k, v in host.items() if k in ("x", "q_idx")}
-        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    if with_e2e:
+        nbytes = lambda ts: int(sum(t.numel() * t.element_size() for t in ts))  # noqa: E731
         ws_e = F.alloc_workspace(ws.numel(), dev)
-        xd, qd = torch.empty_like(d["x"]), torch.empty_like(d["q_idx"])
+        if verify:
+            hin = {k: host[k] for k in ("x_rows", "pos", "view", "rank")}
+            hin.update({"logits": acc["logits"], "kind": acc["kind"], "ref_tok": acc["ref_tok"]})
+            ws_ea = F.alloc_workspace(ws_a.numel(), dev)
+            outs = [out, top1, conf, flags, n_acc]
+        else:
+            # x[Q]: row i of sequence b is x[b, q_idx[b, i]], gathered once on the host
+            qi = host["q_idx"].long()
+            hin = {"x_rows": torch.stack([host["x"][b, qi[b]] for b in range(B)]).contiguous(),
+                   "q_idx": host["q_idx"]}
+            outs = [out]
+        pin = {k: v.pin_memory() for k, v in hin.items()}
+        dbuf = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in pin.items()}
+        outs_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+
+        def e2e_step():
+            for k in pin:
+                dbuf[k].copy_(pin[k], non_blocking=True)
+            if verify:
+                F.fdllm_verify_step(dbuf["x_rows"], dbuf["pos"], dbuf["view"], dbuf["rank"],
+                                    d["w_qkv"], d["k_cache"], d["v_cache"], d["k_side"],
+                                    d["v_side"], out, ws_e, rope_base=rope_base)
+                F.fdllm_accept(dbuf["logits"], dbuf["kind"], dbuf["ref_tok"], dbuf["rank"], top1,
+                               conf, flags, n_acc, ws_ea, eps=0.9, gamma=0.8)
+            else:
+                F.fdllm_fused_step_rows(dbuf["x_rows"], dbuf["q_idx"], d["w_qkv"], d["k_cache"],
+                                        d["v_cache"], out, ws_e, rope_base=rope_base)
+            for oh, o in zip(outs_h, outs):
+                oh.copy_(o, non_blocking=True)
+
         e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(max(3, args.steps // 4))]
         for i in range(args.warmup + len(e2e_ev)):
@@ -339,21 +393,20 @@ def run_ours(args, world, rank, local, cfg=None, name=None, with_e2e=True):
             ev = e2e_ev[i - args.warmup] if i >= args.warmup else None
             if ev:
                 ev[0].record()
-            xd.copy_(pin["x"], non_blocking=True)
-            qd.copy_(pin["q_idx"], non_blocking=True)
-            F.fdllm_fused_step(xd, qd, d["w_qkv"], d["k_cache"], d["v_cache"], out, ws_e,
-                               rope_base=rope_base)
-            out_h.copy_(out, non_blocking=True)
+            e2e_step()
             if ev:
                 ev[1].record()
         torch.cuda.synchronize()
         e2e_ms = F.max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / len(e2e_ev), dev)
-        e2e = {"value": tokens_per_step / (e2e_ms / 1e3), "unit": "query-tokens/s",
-               "h2d_bytes_per_step": int(pin["x"].numel() * pin["x"].element_size()
-                                         + pin["q_idx"].numel() * 4),
-               "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()),
+        e2e = {"value": tokens_per_step / (e2e_ms / 1e3),
+               "unit": "query-tokens/s" if not verify else "query-rows/s",
+               "h2d_bytes_per_step": nbytes(pin.values()),
+               "d2h_bytes_per_step": nbytes(outs_h),
                "ms_per_step": e2e_ms,
-               "path": "pinned host x, q_idx -> fdllm_fused_step -> pinned host out"}
+               "path": ("pinned host x_rows, pos, view, rank, logits, kind, ref_tok -> "
+                        "fdllm_verify_step + fdllm_accept -> pinned host out, top1, conf, flags, "
+                        "n_accept") if verify else
+                       "pinned host x[Q] rows, q_idx -> fdllm_fused_step_rows -> pinned host out"}
 
     # ---------------- roofline of the dominant kernel
     peak, peak_kind = measured_peaks()
@@ -380,9 +433,7 @@ def run_ours(args, world, rank, local, cfg=None, name=None, with_e2e=True):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": mean_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg["dtype"], "data": "synthetic",
-        "config": {"workload": workload_desc(name, cfg),
-                   "l2": "flushed before every timed step (512 MB write)",
-                   "parallelism": f"replicas x{world} (sequences sharded, no collective)"},
+        "config": bench_config(name, cfg, world),
         "hbm_gbs_step": step_bytes / (mean_step / 1e3) / 1e9,
         "step_roofline_frac": step_bytes / (mean_step / 1e3) / 1e9 / peak,
         "step_roofline_frac_nominal": step_bytes / (mean_step / 1e3) / 1e9 / NOMINAL_HBM_GBS,
@@ -464,8 +515,7 @@ def run_reference(args, world, rank):
             "steps": len(per_step), "warmup": min(1, args.warmup), "ms_per_step": mean * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": workload_desc(args.workload, cfg), "l2": "n/a (host)",
-                       "parallelism": "host cores"},
+            "config": bench_config(args.workload, cfg, world),
             "cpu_baseline": {"value": value, "unit": unit, "cores": cpu_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -482,6 +532,13 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=[k for k in W.CONFIGS if k != "tiny_fp32"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end pass")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch B (a smaller case of the same kernels, "
+                         "e.g. for a profiler capture)")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="override the workload's cache length N (the generated block stays "
+                         "at the end; the prompt shrinks)")
     ap.add_argument("--sweep-batch", action="store_true",
                     help="batch scaling study: the single-sequence shape (N = 512 prompt + 512 "
                          "generated, |Q| = 32) at B = 1..64 per GPU, one JSON line per B")
@@ -513,9 +570,9 @@ def main():
                                       "stage_ms": r["stage_ms"], "clocks": r["clocks"],
                                       "config": r["config"]}), flush=True)
             return
-        res = run_ours(args, world, rank, local)
+        cfg, name = workload_with_overrides(args)
+        res = run_ours(args, world, rank, local, cfg=cfg, name=name, with_e2e=not args.no_e2e)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            cfg = W.CONFIGS[args.workload]
             v, reps, units, _ = time_oracle(cfg, float(os.environ.get("FDLLM_ORACLE_BUDGET_S", "15")), 50)
             res["cpu_baseline"] = {
                 "value": v, "unit": res["unit"], "cores": cpu_threads(), "kind": "oracle",

@@ -117,6 +117,17 @@ fdllm_status fdllm_fused_step(int B, int N, int D, int H, int dh, int nq, int dt
                               float rope_base, void* k_cache, void* v_cache, void* out,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* fdllm_fused_step for a caller that holds only the rows the step reads: x_rows
+ * [B, nq, D], row i of sequence b being the hidden state of slot q_idx[b, i]
+ * (what a layer of the same decode step produces, since only the rows of Q are
+ * recomputed).  Everything else, the workspace and the results are those of
+ * fdllm_fused_step; both give the same bits.  A repeated or out-of-range index
+ * sets FDLLM_ERR_BAD_INDEX (repeats: bf16 only). */
+fdllm_status fdllm_fused_step_rows(int B, int N, int D, int H, int dh, int nq, int dtype,
+                                   const void* x_rows, const int32_t* q_idx, const void* w_qkv,
+                                   float rope_base, void* k_cache, void* v_cache, void* out,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
 /* Stage 1 of fdllm_fused_step: gather x[Q], project, rotate, write k,v into the
  * cache and the rotated queries into q_out [B, nq, H, dh] (storage dtype). */
 fdllm_status fdllm_qkv_rope_scatter(int B, int N, int D, int H, int dh, int nq, int dtype,
@@ -209,7 +220,10 @@ fdllm_status fdllm_accept(int B, int R, int V, const float* logits, const int8_t
  *   streams, or from several threads) race on the array: order them.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture. */
+ *   before any stream capture.  The address is kept per device and per
+ *   context: a call made after cudaDeviceReset (or a primary-context reset),
+ *   or with another context current, looks it up again, since the array then
+ *   lives at a new address; the array's contents do not survive a reset. */
 fdllm_status fdllm_accept_noalloc(int B, int R, int V, const float* logits, const int8_t* kind,
                                   const int32_t* ref_tok, const int32_t* rank, float eps,
                                   float gamma, int32_t* top1, float* conf, uint8_t* flags,
@@ -244,6 +258,34 @@ fdllm_status fdllm_track_select(int B, int N, int H, int dh, int nq, int dtype,
                                 const int8_t* q_masked, const int8_t* candidate,
                                 const void* k_cache, int beta_t, int32_t* track, float* mass,
                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Diagnostic: how the bf16 attention of a step with these shapes spreads its
+ * work over the current device's SMs (the choice depends only on the shapes and
+ * the device).  rows = nq (fused step) or R (verify pass, verify = 1).
+ *   1  persistent stream-K: one CTA per SM, each an equal contiguous range of
+ *      (item, 128-key tile) units; an item split between CTAs is merged by its
+ *      last contributor;
+ *   2  one CTA per whole (sequence, head, query chunk) item, no merge;
+ *   3  a thread-block cluster per item, merged through distributed shared
+ *      memory; *cluster_size (host pointer, may be NULL) gets its CTA count.
+ *  -1  shapes the bf16 attention does not run.
+ * Launches nothing and allocates nothing. */
+int fdllm_attention_split(int B, int N, int H, int dh, int rows, int S_max, int verify,
+                          int* cluster_size);
+
+/* Diagnostic: runs the bounded wait that every kernel of this library uses on
+ * its mbarriers, against an mbarrier that nothing completes, so that its
+ * timeout path can be checked without a fault or a hang.  One CTA: one thread
+ * waits with limit_ns (1 us .. 2 s, the kernels' own limit; else
+ * FDLLM_ERR_INVALID_ARG) and must give up, recording FDLLM_ERR_TIMEOUT in the
+ * status word; a second thread then waits on the same barrier and must return
+ * at once, as every later wait of a kernel does after a timeout.
+ *   workspace: >= 288 bytes, 256-byte aligned, status word zero.  Results at
+ *   byte 256, four uint64: first wait completed (0/1), its duration in ns,
+ *   second wait completed (0/1), its duration in ns.
+ * Read the status with fdllm_get_status; zero the workspace before reusing it. */
+fdllm_status fdllm_bounded_wait_selftest(uint64_t limit_ns, void* workspace,
+                                         size_t workspace_bytes, void* stream);
 
 /* Number of kernels this library has launched in this process (a diagnostic
  * counter, incremented on the host at every launch; never reset). */

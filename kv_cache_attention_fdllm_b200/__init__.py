@@ -11,13 +11,16 @@ lib()  # fail loudly at import when the CUDA library is missing
 
 from .api import (ERR_BAD_INDEX, ERR_CUDA, ERR_INVALID_ARG, ERR_TIMEOUT, ERR_UNSUPPORTED,  # noqa: E402
                   ERR_WORKSPACE, FLAG_ACCEPT, FLAG_COMMIT, FLAG_PASS, OK, FdllmError,
-                  alloc_workspace, fdllm_accept, fdllm_accept_noalloc,
+                  SPLIT_CLUSTERS, SPLIT_STREAM_K, SPLIT_WHOLE_ITEMS,
+                  alloc_workspace, fdllm_accept, fdllm_accept_noalloc, fdllm_attention_split,
+                  fdllm_bounded_wait_selftest,
                   fdllm_accept_workspace_bytes, fdllm_attend,
-                  fdllm_fused_step, fdllm_fused_step_workspace_bytes, fdllm_get_status,
+                  fdllm_fused_step, fdllm_fused_step_rows, fdllm_fused_step_workspace_bytes,
+                  fdllm_get_status,
                   fdllm_qkv_rope_scatter, fdllm_verify_attend, fdllm_verify_qkv_rope_scatter,
                   fdllm_track_select, fdllm_verify_step, fdllm_verify_step_workspace_bytes)
 
 from .shard import max_over_ranks, rank_sequences  # noqa: E402
 
-__all__ = [n for n in dir() if n.startswith(("fdllm_", "FLAG_", "ERR_"))] + [
+__all__ = [n for n in dir() if n.startswith(("fdllm_", "FLAG_", "ERR_", "SPLIT_"))] + [
     "OK", "FdllmError", "alloc_workspace", "lib", "LIB_PATH", "max_over_ranks", "rank_sequences"]

@@ -20,6 +20,8 @@ SIGNATURES = {
     "fdllm_accept_workspace_bytes": (_c_size, [_c_int] * 3),
     "fdllm_fused_step": (_c_int, [_c_int] * 7 + [_vp, _vp, _vp, _c_float, _vp, _vp, _vp, _vp,
                                                  _c_size, _vp]),
+    "fdllm_fused_step_rows": (_c_int, [_c_int] * 7 + [_vp, _vp, _vp, _c_float, _vp, _vp, _vp,
+                                                      _vp, _c_size, _vp]),
     "fdllm_qkv_rope_scatter": (_c_int, [_c_int] * 7 + [_vp, _vp, _vp, _c_float, _vp, _vp, _vp,
                                                        _vp, _c_size, _vp]),
     "fdllm_attend": (_c_int, [_c_int] * 6 + [_vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
@@ -36,6 +38,8 @@ SIGNATURES = {
                                                      _vp, _vp, _vp, _vp, _vp]),
     "fdllm_track_select": (_c_int, [_c_int] * 6 + [_vp, _vp, _vp, _c_int, _vp, _vp, _vp, _c_size,
                                                     _vp]),
+    "fdllm_attention_split": (_c_int, [_c_int] * 7 + [_vp]),
+    "fdllm_bounded_wait_selftest": (_c_int, [ctypes.c_uint64, _vp, _c_size, _vp]),
     "fdllm_launch_count": (ctypes.c_uint64, []),
     "fdllm_get_status": (_c_int, [_vp, _vp]),
 }

@@ -125,6 +125,28 @@ def fdllm_fused_step(x, q_idx, w_qkv, k_cache, v_cache, out, workspace, rope_bas
     return out
 
 
+def fdllm_fused_step_rows(x_rows, q_idx, w_qkv, k_cache, v_cache, out, workspace,
+                          rope_base=10000.0, stream=None):
+    """fdllm_fused_step with the rows x[Q] given packed, x_rows [B, nq, D]."""
+    _need(x_rows, "x_rows")
+    B, nq, D = x_rows.shape
+    _need(k_cache, "k_cache")
+    H, N, dh = k_cache.shape[1], k_cache.shape[2], k_cache.shape[3]
+    dt, dev = x_rows.dtype, x_rows.device
+    _need(q_idx, "q_idx", torch.int32, (B, nq), dev)
+    _need(w_qkv, "w_qkv", dt, (3 * H * dh, D), dev)
+    _need(k_cache, "k_cache", dt, (B, H, N, dh), dev)
+    _need(v_cache, "v_cache", dt, (B, H, N, dh), dev)
+    _need(out, "out", dt, (B, nq, H * dh), dev)
+    _need(workspace, "workspace", torch.uint8, None, dev)
+    st = lib().fdllm_fused_step_rows(B, N, D, H, dh, nq, _dtype_code(x_rows), _p(x_rows),
+                                     _p(q_idx), _p(w_qkv), float(rope_base), _p(k_cache),
+                                     _p(v_cache), _p(out), _p(workspace), workspace.numel(),
+                                     _stream(stream, dev))
+    _check(st, "fdllm_fused_step_rows")
+    return out
+
+
 def fdllm_qkv_rope_scatter(x, q_idx, w_qkv, k_cache, v_cache, q_out, workspace,
                            rope_base=10000.0, stream=None):
     B, N, D, H, dh, nq = _check_fused(x, q_idx, w_qkv, k_cache, v_cache)
@@ -299,6 +321,33 @@ def fdllm_accept_noalloc(logits, kind, ref_tok, rank, top1, conf, flags, n_accep
                                     _p(n_accept), _stream(stream, dev))
     _check(st, "fdllm_accept_noalloc")
     return top1, conf, flags, n_accept
+
+
+SPLIT_STREAM_K, SPLIT_WHOLE_ITEMS, SPLIT_CLUSTERS = 1, 2, 3
+
+
+def fdllm_attention_split(B, N, H, dh, rows, S_max=0, verify=False):
+    """(split, cluster_size): how the bf16 attention spreads these shapes over the
+    current device (SPLIT_STREAM_K, SPLIT_WHOLE_ITEMS or SPLIT_CLUSTERS; -1 if
+    it does not run them).  A diagnostic: launches nothing."""
+    cs = ctypes.c_int(0)
+    mode = lib().fdllm_attention_split(B, N, H, dh, rows, S_max, int(bool(verify)),
+                                       ctypes.byref(cs))
+    return int(mode), int(cs.value)
+
+
+def fdllm_bounded_wait_selftest(limit_ns, workspace, stream=None):
+    """Runs the kernels' bounded mbarrier wait against a barrier nothing completes
+    (see include/fdllm.h).  Returns the four result words (first wait completed,
+    its ns, second wait completed, its ns) after synchronising the stream; the
+    status word is left for fdllm_get_status."""
+    _need(workspace, "workspace", torch.uint8, None, None)
+    st = lib().fdllm_bounded_wait_selftest(int(limit_ns), _p(workspace), workspace.numel(),
+                                           _stream(stream, workspace.device))
+    _check(st, "fdllm_bounded_wait_selftest")
+    torch.cuda.current_stream(workspace.device).synchronize() if stream is None else \
+        stream.synchronize()
+    return [int(v) for v in workspace[256:288].view(torch.int64).cpu().tolist()]
 
 
 def fdllm_get_status(workspace, stream=None) -> int:

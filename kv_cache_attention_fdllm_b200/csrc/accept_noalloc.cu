@@ -10,9 +10,12 @@
 //
 // The array is file-scope and static: every GPU that loads the library holds
 // it until the process exits.  Host code only sees a host-side stand-in under
-// its name, so the device address is looked up once per device with
-// cudaGetSymbolAddress (on the first call, with that device current) and that
-// address is what the kernel receives.
+// its name, so the device address is looked up with cudaGetSymbolAddress, with
+// the device current, once per device and context (the first call there), and
+// that address is what the kernel receives.  The lookup is keyed on the
+// current context's unique id: after a cudaDeviceReset, or with another
+// context current on the same device, the module is loaded anew at another
+// address, and the next call looks it up again.
 #include <mutex>
 
 #include "common.cuh"
@@ -25,22 +28,65 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_accept_scratch[kScratchBytes];
 
-std::mutex g_scratch_mu;
-void* g_scratch_dev_ptr[kMaxDevices];  // device address of g_accept_scratch, per device
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
-// Device address of the scratch array on the current device (set-up on first use).
+struct DriverFns {
+  CtxGetCurrentFn get_current = nullptr;
+  CtxGetIdFn get_id = nullptr;
+};
+
+const DriverFns& driver_fns() {
+  static DriverFns f;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      f.get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      f.get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  return f;
+}
+
+// Unique id of the calling thread's current context, 0 when there is none yet.
+unsigned long long current_context_id() {
+  const DriverFns& f = driver_fns();
+  if (!f.get_current || !f.get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (f.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  return f.get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+struct ScratchAddr {
+  unsigned long long ctx_id;  // context the address belongs to (0: none cached)
+  void* ptr;
+};
+
+std::mutex g_scratch_mu;
+ScratchAddr g_scratch[kMaxDevices];  // device address of g_accept_scratch, per device
+
+// Device address of the scratch array in the current context (set-up on the
+// first call on each device and context).
 fdllm_status scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FDLLM_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return FDLLM_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_dev_ptr[dev]) {
+  const unsigned long long id = current_context_id();
+  if (id == 0 || g_scratch[dev].ctx_id != id || !g_scratch[dev].ptr) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_accept_scratch);
     if (e != cudaSuccess || p == nullptr) return FDLLM_ERR_CUDA;
-    g_scratch_dev_ptr[dev] = p;
+    // the lookup made the device's primary context current if none was
+    g_scratch[dev].ctx_id = current_context_id();
+    g_scratch[dev].ptr = p;
   }
-  *out = g_scratch_dev_ptr[dev];
+  *out = g_scratch[dev].ptr;
   return FDLLM_OK;
 }
 

@@ -83,10 +83,10 @@ fdllm_status run_proj(int B, int N, int D, int H, int dh, int rows, int S_max, i
                       int dtype, const void* x, const int32_t* idx, const int8_t* view,
                       const void* w, float rope_base, void* k_cache, void* v_cache,
                       void* k_side, void* v_side, void* q_out, void* ws, const Layout& L,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, int packed = 0) {
   ProjArgs a{};
   a.B = B; a.N = N; a.D = D; a.H = H; a.dh = dh; a.rows_per_seq = rows; a.S_max = S_max;
-  a.verify = verify; a.dtype = dtype;
+  a.verify = verify; a.dtype = dtype; a.packed = verify ? 1 : packed;
   a.x = x; a.idx = idx; a.view = view; a.w = w;
   a.log2_base = log2((double)rope_base);
   a.k_cache = k_cache; a.v_cache = v_cache; a.k_side = k_side; a.v_side = v_side;
@@ -238,6 +238,27 @@ fdllm_status fdllm_fused_step(int B, int N, int D, int H, int dh, int nq, int dt
                   v_cache, nullptr, nullptr, out, workspace, L, s);
 }
 
+fdllm_status fdllm_fused_step_rows(int B, int N, int D, int H, int dh, int nq, int dtype,
+                                   const void* x_rows, const int32_t* q_idx, const void* w_qkv,
+                                   float rope_base, void* k_cache, void* v_cache, void* out,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("fdllm_fused_step_rows");
+  fdllm_status st = check_shape(B, N, D, H, dh, nq, dtype);
+  if (st != FDLLM_OK) return st;
+  if (!(rope_base > 0.f)) return FDLLM_ERR_INVALID_ARG;
+  const Layout L = step_layout(B, N, D, H, dh, nq, 0, 0, dtype);
+  if ((st = check_ws(workspace, workspace_bytes, L.total)) != FDLLM_OK) return st;
+  if (B * nq == 0) return FDLLM_OK;
+  if (!all_aligned({x_rows, q_idx, w_qkv, k_cache, v_cache, out})) return FDLLM_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* q = ws_at(workspace, L.q_off);
+  st = run_proj(B, N, D, H, dh, nq, 0, 0, dtype, x_rows, q_idx, nullptr, w_qkv, rope_base,
+                k_cache, v_cache, nullptr, nullptr, q, workspace, L, s, /*packed=*/1);
+  if (st != FDLLM_OK) return st;
+  return run_attn(B, N, H, dh, nq, 0, 0, 0, dtype, q, nullptr, nullptr, nullptr, k_cache,
+                  v_cache, nullptr, nullptr, out, workspace, L, s);
+}
+
 fdllm_status fdllm_verify_qkv_rope_scatter(int B, int N, int D, int H, int dh, int R, int S_max,
                                            int dtype, const void* x_rows, const int32_t* pos,
                                            const int8_t* view, const void* w_qkv,
@@ -363,6 +384,28 @@ fdllm_status fdllm_track_select(int B, int N, int H, int dh, int nq, int dtype,
                 : reinterpret_cast<float*>(ws_at(
                       workspace, L.track_off + align_up((size_t)B * H * N * sizeof(float), 256)));
   return from_cuda(launch_track(a, static_cast<cudaStream_t>(stream)));
+}
+
+int fdllm_attention_split(int B, int N, int H, int dh, int rows, int S_max, int verify,
+                          int* cluster_size) {
+  int cs = 0;
+  int mode = -1;
+  if (check_shape(B, N, 64, H, dh, rows, FDLLM_BF16) == FDLLM_OK && (verify == 0 || verify == 1) &&
+      S_max >= 0 && !(verify && rows > kMaxVerifyRows))
+    mode = attn_tc_split(B, N, H, dh, rows, verify ? S_max : 0, verify, &cs);
+  if (cluster_size) *cluster_size = mode == 3 ? cs : 0;
+  return mode;
+}
+
+fdllm_status fdllm_bounded_wait_selftest(uint64_t limit_ns, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  if (limit_ns < 1000 || limit_ns > kWaitLimitNs) return FDLLM_ERR_INVALID_ARG;
+  fdllm_status st = check_ws(workspace, workspace_bytes, kWsHeaderBytes + 32);
+  if (st != FDLLM_OK) return st;
+  return from_cuda(launch_bounded_wait_selftest(
+      reinterpret_cast<int*>(workspace), limit_ns,
+      reinterpret_cast<unsigned long long*>(ws_at(workspace, kWsHeaderBytes)),
+      static_cast<cudaStream_t>(stream)));
 }
 
 fdllm_status fdllm_get_status(void* workspace, void* stream) {

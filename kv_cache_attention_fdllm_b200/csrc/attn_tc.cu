@@ -54,6 +54,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kThresh = 8.f;  // lazy rescale threshold (log2 units)
 constexpr int kMaxRows = 512;   // verify rows per sequence held in shared memory
 constexpr int kL2PrefetchTiles = 4;  // cache tiles per CTA warmed in L2 before the dependency wait
+// work splits (the values fdllm_attention_split reports)
+constexpr int kSplitStreamK = 1, kSplitWholeItems = 2, kSplitClusters = 3;
 
 struct AttnTcParams {
   int B, N, H, rows, S_max, causal;
@@ -1022,17 +1024,35 @@ int max_clusters(int cs, size_t smem_bytes) {
   return cache[cs];
 }
 
+// The work split a launch of this plan takes (kSplit*), after the kernel's
+// shared-memory limit is raised; *cs_out gets the cluster size (0 without).
+// Cluster mode only when every item's cluster fits in one wave.
 template <int NQ, int DH, bool VERIFY>
-cudaError_t launch_t(const AttnArgs& a, const AttnPlan& q, AttnTcParams prm, const CUtensorMap* maps,
-                     cudaStream_t stream) {
+cudaError_t resolve_split(const AttnPlan& q, int* mode, int* cs_out) {
   auto kern = attn_tc_kernel<NQ, DH, VERIFY>;
   const size_t smem_max = q.smem_bytes > q.smem_cl ? q.smem_bytes : q.smem_cl;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem_max);
   if (e != cudaSuccess) return e;
-  // cluster mode only when every item's cluster fits in one wave
   int cs = q.cs;
   while (cs >= 2 && max_clusters<NQ, DH, VERIFY>(cs, q.smem_cl) < q.items) --cs;
+  if (cs >= 2) {
+    *mode = kSplitClusters;
+    *cs_out = cs;
+  } else {
+    *mode = q.whole_items ? kSplitWholeItems : kSplitStreamK;
+    *cs_out = 0;
+  }
+  return cudaSuccess;
+}
+
+template <int NQ, int DH, bool VERIFY>
+cudaError_t launch_t(const AttnArgs& a, const AttnPlan& q, AttnTcParams prm, const CUtensorMap* maps,
+                     cudaStream_t stream) {
+  auto kern = attn_tc_kernel<NQ, DH, VERIFY>;
+  int mode = 0, cs = 0;
+  cudaError_t e = resolve_split<NQ, DH, VERIFY>(q, &mode, &cs);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(Threads<NQ>::kAll);
   cfg.stream = stream;
@@ -1041,7 +1061,7 @@ cudaError_t launch_t(const AttnArgs& a, const AttnPlan& q, AttnTcParams prm, con
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cs >= 2) {
+  if (mode == kSplitClusters) {
     attr[1].id = cudaLaunchAttributeClusterDimension;
     attr[1].val.clusterDim.x = cs;
     attr[1].val.clusterDim.y = 1;
@@ -1053,7 +1073,7 @@ cudaError_t launch_t(const AttnArgs& a, const AttnPlan& q, AttnTcParams prm, con
     prm.nk = q.nk_cl;
     prm.nv = q.nv_cl;
     prm.nqbuf = 1;
-  } else if (q.whole_items) {
+  } else if (mode == kSplitWholeItems) {
     // grid = items: the unit split gives every CTA exactly one whole item
     cfg.gridDim = dim3((unsigned)q.items);
     cfg.dynamicSmemBytes = q.smem_cl;
@@ -1081,6 +1101,26 @@ size_t attn_tc_workspace_bytes(int B, int N, int H, int dh, int rows, int S_max,
   if (B * rows <= 0) return 256;
   const AttnPlan q = plan(B, N, H, dh, rows, S_max, verify, num_sms);
   return q.partial_bytes + q.counter_bytes;
+}
+
+int attn_tc_split(int B, int N, int H, int dh, int rows, int S_max, int verify, int* cs) {
+  *cs = 0;
+  if (B * rows <= 0 || (verify && rows > kMaxRows)) return -1;
+  const AttnPlan q = plan(B, N, H, dh, rows, S_max, verify, device_sm_count());
+  int mode = -1;
+  cudaError_t e = cudaErrorInvalidValue;
+#define FDLLM_ATTN_SPLIT(NQv, DHv)                                                           \
+  if (q.NQ == NQv && dh == DHv)                                                             \
+    e = verify ? resolve_split<NQv, DHv, true>(q, &mode, cs)                                \
+               : resolve_split<NQv, DHv, false>(q, &mode, cs);
+  FDLLM_ATTN_SPLIT(16, 64)
+  FDLLM_ATTN_SPLIT(32, 64)
+  FDLLM_ATTN_SPLIT(64, 64)
+  FDLLM_ATTN_SPLIT(16, 128)
+  FDLLM_ATTN_SPLIT(32, 128)
+  FDLLM_ATTN_SPLIT(64, 128)
+#undef FDLLM_ATTN_SPLIT
+  return e == cudaSuccess ? mode : -1;
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {

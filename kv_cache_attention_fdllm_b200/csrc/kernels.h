@@ -36,12 +36,14 @@ cudaError_t launch_accept(const AcceptArgs& a, cudaStream_t stream);
 
 // ----------------------------------------------------------------- projection
 // Rows of the projection: token m of sequence b = m / rows_per_seq.
-//   fused  (verify == 0): x row (b, q_idx[m]); RoPE position and cache slot q_idx[m].
-//   verify (verify == 1): x_rows row m; position pos[m]; view[m] chooses the
-//                         destination (0/1: cache slot pos[m]; 2: side slot).
+//   fused  (verify == 0): RoPE position and cache slot q_idx[m]; the input row
+//                         is x row (b, q_idx[m]), or row m when packed.
+//   verify (verify == 1): x_rows row m (always packed); position pos[m]; view[m]
+//                         chooses the destination (0/1: cache slot pos[m]; 2: side slot).
 struct ProjArgs {
   int B, N, D, H, dh, rows_per_seq, S_max, verify, dtype;
-  const void* x;           // fused: [B, N, D]; verify: [B, R, D]
+  int packed;              // x holds the rows themselves, [B, rows, D]
+  const void* x;           // gathered: [B, N, D]; packed: [B, rows, D]
   const int32_t* idx;      // fused: q_idx [B, nq]; verify: pos [B, R]
   const int8_t* view;      // verify only
   const void* w;           // [3E, D]
@@ -109,6 +111,15 @@ cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t stream);
 size_t attn_tc_workspace_bytes(int B, int N, int H, int dh, int rows, int S_max, int verify,
                                int num_sms);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream);
+// The work split launch_attn_tc takes for these shapes on the current device:
+// 1 persistent stream-K, 2 one CTA per whole item, 3 clusters of *cs CTAs per
+// item; -1 for shapes it does not run.
+int attn_tc_split(int B, int N, int H, int dh, int rows, int S_max, int verify, int* cs);
+
+// ----------------------------------------------------------------- diagnostics
+// result[0..3]: first wait completed (0/1), its ns; second wait completed, its ns
+cudaError_t launch_bounded_wait_selftest(int* status, uint64_t limit_ns,
+                                         unsigned long long* result, cudaStream_t stream);
 
 // ----------------------------------------------------------------- helpers
 int device_sm_count();

@@ -21,10 +21,11 @@ constexpr int kTK = 32;  // reduction chunk
 template <typename T>
 __device__ __forceinline__ const T* proj_row(const ProjArgs& a, int m) {
   const T* x = static_cast<const T*>(a.x);
-  if (a.verify) return x + (size_t)m * a.D;
-  const int b = m / a.rows_per_seq;
   const int j = a.idx[m];
+  if (a.verify) return x + (size_t)m * a.D;
   if (j < 0 || j >= a.N) return nullptr;
+  if (a.packed) return x + (size_t)m * a.D;
+  const int b = m / a.rows_per_seq;
   return x + ((size_t)b * a.N + j) * a.D;
 }
 

@@ -56,6 +56,7 @@ constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
 
 struct ProjTcParams {
   int M, F, D, E, N, H, dh, rows_per_seq, S_max, verify;
+  int check_repeats;   // report a repeated index (packed fused rows; the prep kernel does it otherwise)
   int BN, n_tt, tiles, nks, subs, nsub_total, nstage;
   long long total_units;
   const int32_t* idx;
@@ -319,6 +320,13 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             slot = in_range ? ps : -1;
           }
         }
+        // Q is a set: a packed fused row repeating an earlier row's slot is
+        // reported once, by the first feature tile
+        if (p.check_repeats && ft == 0 && m < p.M) {
+          const int ps = p.idx[m];
+          for (int r = (m / p.rows_per_seq) * p.rows_per_seq; r < m; ++r)
+            if (p.idx[r] == ps) set_status(p.status, FDLLM_ERR_BAD_INDEX);
+        }
         tok_slot[n] = slot;
         tok_flag[n] = flag;
         tok_b[n] = m < p.M ? m / p.rows_per_seq : 0;
@@ -563,8 +571,10 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream) {
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
       return cudaErrorInvalidValue;
   }
-  // X: the packed verify rows, or x[Q] packed into the workspace by the prep kernel
-  const void* xsrc = a.verify ? a.x : static_cast<const void*>(xq);
+  // X: rows the caller packed (verify rows, or fused rows given as x[Q]), or
+  // x[Q] packed into the workspace by the prep kernel
+  const bool packed = a.verify || a.packed;
+  const void* xsrc = packed ? a.x : static_cast<const void*>(xq);
   {
     const uint64_t dims[2] = {(uint64_t)a.D, (uint64_t)M};
     const uint64_t strides[1] = {(uint64_t)a.D * 2};
@@ -576,6 +586,7 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream) {
   ProjTcParams p{};
   p.M = M; p.F = F; p.D = a.D; p.E = E; p.N = a.N; p.H = a.H; p.dh = a.dh;
   p.rows_per_seq = a.rows_per_seq; p.S_max = a.S_max; p.verify = a.verify;
+  p.check_repeats = (!a.verify && a.packed) ? 1 : 0;
   p.BN = q.BN; p.n_tt = q.n_tt; p.tiles = q.tiles; p.nks = q.nks; p.subs = q.subs;
   p.nsub_total = q.nsub_total; p.nstage = q.nstage; p.total_units = q.total_units;
   p.idx = a.idx; p.view = a.view; p.log2_base = a.log2_base;
@@ -589,8 +600,8 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream) {
   p.tile_cnt = reinterpret_cast<unsigned*>(ws + q.partial_bytes);
 
   cudaError_t e;
-  if (!a.verify) {
-    // the fused step gathers x[Q] into a packed operand; verify rows arrive packed
+  if (!packed) {
+    // the fused step gathers x[Q] into a packed operand
     proj_prep_kernel<<<M, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.x), a.idx, a.N,
                                             a.D, a.rows_per_seq, xq, a.status);
     count_launches(1);

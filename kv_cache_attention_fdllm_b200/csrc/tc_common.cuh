@@ -56,10 +56,11 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs (or at once when *abort is already set): then records
-// FDLLM_ERR_TIMEOUT, sets *abort and returns false so the caller can leave.
+// limit_ns without completion (or at once when *abort is already set): then
+// records FDLLM_ERR_TIMEOUT, sets *abort and returns false so the caller can
+// leave.  Every kernel waits with the default limit.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* status) {
+                                          int* status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = 0;
   for (uint32_t spin = 1;; ++spin) {
@@ -69,7 +70,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       const uint64_t now = global_ns();
       if (t0 == 0) {
         t0 = now;
-      } else if (now - t0 > kWaitLimitNs) {
+      } else if (now - t0 > limit_ns) {
         *abort = 1;
         set_status(status, FDLLM_ERR_TIMEOUT);
         return false;

@@ -119,7 +119,17 @@ def next_tracked(ranked, decoded, beta_t):
     return torch.gather(ranked, 1, first).contiguous()
 
 
-def run(cfg: LoopConfig, device="cuda") -> dict:
+def _cpu(t):
+    return t.detach().to("cpu", copy=True)
+
+
+def run(cfg: LoopConfig, device="cuda", trace: dict | None = None) -> dict:
+    """Decodes the generated block.  With a dict as `trace`, the first step's
+    calls record their inputs and results in it (CPU copies): the draft pass of
+    layer 0 and of the middle layer ("draft"), the tracked-set selection
+    ("track"), the epsilon split ("split"), the verify pass of layer 0
+    ("verify"), the gamma acceptance ("gamma") and the sets the step ends with
+    ("sets"), so that each call can be replayed on the same inputs."""
     dev = torch.device(device)
     gen = torch.Generator(device=dev)
     gen.manual_seed(cfg.seed)
@@ -158,20 +168,34 @@ def run(cfg: LoopConfig, device="cuda") -> dict:
         masks_left = (~decoded).sum(dim=1)
         if int(masks_left.max()) == 0:
             break  # a finished sequence rides along with an all-decoded Q until then
+        rec = trace if (trace is not None and steps == 0) else None
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ev0.record()
         q_idx, q_masked, front = query_set(decoded, T, cfg.beta_m)
+        if rec is not None:
+            rec.update(draft={}, decoded_before=_cpu(decoded), T=_cpu(T), q_idx=_cpu(q_idx),
+                       q_masked=_cpu(q_masked), front=_cpu(front), W=[_cpu(w) for w in W])
 
         # draft pass over the layers; the tracked set comes from the middle layer
         x = x0.clone()
         rows = q_idx.long()
         bidx = torch.arange(B, device=dev).unsqueeze(1)
         for l in range(cfg.L):
+            keep = rec is not None and l in (0, cfg.L // 2)
+            if keep:
+                rec["draft"][l] = {"x": _cpu(x), "k_in": _cpu(K[l]), "v_in": _cpu(V[l])}
             F.fdllm_fused_step(x, q_idx, W[l], K[l], V[l], out, ws)
+            if keep:
+                rec["draft"][l].update(out=_cpu(out), k_out=_cpu(K[l]), v_out=_cpu(V[l]))
             if l == cfg.L // 2:
                 cand = decoded.clone()
                 cand.scatter_(1, front.long(), q_masked[:, cfg.beta_t:].bool() | torch.gather(cand, 1, front.long()))
-                F.fdllm_track_select(q_masked, cand.to(torch.int8).contiguous(), K[l], track, ws)
+                cand8 = cand.to(torch.int8).contiguous()
+                mass = torch.empty((B, N), dtype=torch.float32, device=dev) if rec is not None else None
+                F.fdllm_track_select(q_masked, cand8, K[l], track, ws, mass=mass)
+                if rec is not None:
+                    rec["track"] = {"layer": l, "candidate": _cpu(cand8), "track": _cpu(track),
+                                    "mass": _cpu(mass)}
             x[bidx, rows] = x[bidx, rows] + out
         # epsilon split of the masked rows (stand-in LM head: synthetic logits)
         R1 = cfg.beta_m
@@ -183,6 +207,9 @@ def run(cfg: LoopConfig, device="cuda") -> dict:
         n_acc = torch.empty((B,), dtype=torch.int32, device=dev)
         F.fdllm_accept(logits, kind, None, None, top1, conf, flags, n_acc, ws_a, eps=cfg.eps,
                        gamma=cfg.gamma)
+        if rec is not None:
+            rec["split"] = {"logits": _cpu(logits), "kind": _cpu(kind), "top1": _cpu(top1),
+                            "conf": _cpu(conf), "flags": _cpu(flags)}
         valid = q_masked[:, cfg.beta_t:].bool()
         commit = ((flags & F.FLAG_COMMIT) != 0) & valid
         # exploratory rows in decoding order (confidence descending)
@@ -209,9 +236,16 @@ def run(cfg: LoopConfig, device="cuda") -> dict:
             out_v = torch.empty((B, R, H * dh), dtype=bf, device=dev)
             for l in range(cfg.L):
                 x_rows = xv[bidx, rv].contiguous()
+                if rec is not None and l == 0:
+                    rec["verify"] = {"x_rows": _cpu(x_rows), "pos": _cpu(pos), "view": _cpu(view),
+                                     "rank": _cpu(rank), "k_in": _cpu(K[l]), "v_in": _cpu(V[l]),
+                                     "ks_in": _cpu(KS[l]), "vs_in": _cpu(VS[l])}
                 # the first n_s side slots take the mask view; the rest stay unused
                 F.fdllm_verify_step(x_rows, pos, view, rank, W[l], K[l], V[l], KS[l], VS[l], out_v,
                                     ws_v, causal_cross=cfg.causal_cross)
+                if rec is not None and l == 0:
+                    rec["verify"].update(out=_cpu(out_v), k_out=_cpu(K[l]), v_out=_cpu(V[l]),
+                                         ks_out=_cpu(KS[l]), vs_out=_cpu(VS[l]))
                 xv[bidx, rv] = xv[bidx, rv] + out_v
             # mask-view predictions agree with the draft with probability 0.8
             d_tok = torch.gather(draft_tok, 1, pick)
@@ -226,6 +260,10 @@ def run(cfg: LoopConfig, device="cuda") -> dict:
             F.fdllm_accept(lg_v, kind_v, d_tok.contiguous(), rank_v, t1, c1, f1, n_acc, ws_a,
                            eps=cfg.eps, gamma=cfg.gamma)
             acc_v = (f1 & F.FLAG_ACCEPT) != 0
+            if rec is not None:
+                rec["gamma"] = {"logits": _cpu(lg_v), "kind": _cpu(kind_v), "ref_tok": _cpu(d_tok),
+                                "rank": _cpu(rank_v), "top1": _cpu(t1), "conf": _cpu(c1),
+                                "flags": _cpu(f1), "n_accept": _cpu(n_acc), "s_pos": _cpu(s_pos)}
             newly.scatter_(1, s_pos.long(), acc_v | torch.gather(newly, 1, s_pos.long()))
         # progress policy: at least the most confident masked row per sequence
         none = ~newly.any(dim=1)
@@ -236,6 +274,9 @@ def run(cfg: LoopConfig, device="cuda") -> dict:
         newly &= ~decoded
         decoded |= newly
         T = next_tracked(track, decoded, cfg.beta_t)
+        if rec is not None:
+            rec["sets"] = {"newly": _cpu(newly), "progress_forced": _cpu(none),
+                           "decoded": _cpu(decoded), "T_next": _cpu(T), "n_s": n_s}
         ev1.record()
         torch.cuda.synchronize()
         for w in (ws, ws_v, ws_a):

@@ -64,6 +64,25 @@ def check_cache_update(k_gpu, k_in, k_ref, q_idx, dtype, what):
                      f"{what} written slots, sequence {b}")
 
 
+def check_outside_q_on_device(k_dev, k_in, idx, what, written_mask=None):
+    """Every slot of every sequence outside its written set is bit-identical to
+    the input, compared on the device.  k_dev: the cache after the call (CUDA,
+    [B, H, N, dh]); k_in: the input cache (CPU); idx: int [B, n] the written
+    slots (entries outside [0, N) ignored), or written_mask: bool [B, N]."""
+    B, H, N, dh = k_dev.shape
+    if written_mask is None:
+        written_mask = np.zeros((B, N), bool)
+        ix = np.asarray(idx)
+        for b in range(B):
+            ok = ix[b][(ix[b] >= 0) & (ix[b] < N)]
+            written_mask[b, ok] = True
+    for b in range(B):
+        keep = torch.from_numpy(~written_mask[b]).to(k_dev.device)
+        ref = k_in[b].to(k_dev.device)
+        assert torch.equal(k_dev[b][:, keep], ref[:, keep]), \
+            f"{what}: a slot outside the written set changed in sequence {b}"
+
+
 def run_fused_gpu(F, inp_dev: dict, rope_base: float):
     x = inp_dev["x"]
     B, N, D = x.shape

@@ -5,7 +5,8 @@ import torch
 
 import oracle as O
 import workloads as W
-from parity import (assert_close, check_cache_update, dtype_name, oracle_fused, run_fused_gpu)
+from parity import (assert_close, check_cache_update, check_outside_q_on_device, dtype_name,
+                    oracle_fused, run_fused_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -23,6 +24,9 @@ def _check_fused(F, inp, rope_base=10000.0, seqs_for_oracle=None, inp_oracle=Non
     k_in, v_in = inp["k_cache"].clone(), inp["v_cache"].clone()
     out, ws, st = run_fused_gpu(F, dev, rope_base)
     assert st == F.OK, f"device status {st}"
+    # every sequence, sampled for the oracle or not: slots outside Q bit-identical
+    check_outside_q_on_device(dev["k_cache"], inp["k_cache"], inp["q_idx"], "k_cache")
+    check_outside_q_on_device(dev["v_cache"], inp["v_cache"], inp["q_idx"], "v_cache")
     dt = dtype_name(inp["x"])
     H, dh = inp["k_cache"].shape[1], inp["k_cache"].shape[3]
     sel = list(range(inp["x"].shape[0])) if seqs_for_oracle is None else list(seqs_for_oracle)
@@ -72,6 +76,54 @@ def test_ragged_shapes(F, dtype, dh, shape):
     B, N, D, H, nq = shape
     inp = W.random_fused(B, N, D, H, dh, nq=nq, dtype=dtype, seed=hash((shape, dh)) % 1000)
     _check_fused(F, inp)
+
+
+# (B, N, D, H, dh, nq, work split the attention must take on 148 SMs); items =
+# B * H * query chunks of up to 64 rows.  Whole-item mode takes SMs < items <=
+# 2 SMs when its two waves are no slower than stream-K; stream-K takes the rest
+# above SMs / 2.
+SPLIT_SHAPES = [
+    pytest.param(5, 1000, 128, 32, 64, 20, "whole", id="whole-160items-nq32-dh64"),
+    pytest.param(12, 700, 128, 16, 128, 12, "whole", id="whole-192items-nq16-dh128"),
+    pytest.param(8, 1024, 128, 32, 128, 32, "whole", id="whole-256items-nq32-dh128"),
+    pytest.param(3, 900, 128, 32, 128, 40, "stream", id="streamk-96items-nq64-dh128"),
+    pytest.param(12, 600, 128, 32, 64, 30, "stream", id="streamk-384items-nq32-dh64"),
+    pytest.param(2, 800, 128, 32, 64, 100, "stream", id="streamk-128items-2chunks-dh64"),
+    pytest.param(16, 1024, 128, 32, 128, 32, "stream", id="streamk-512items-nq32-dh128"),
+]
+_SPLIT_CODE = {"stream": 1, "whole": 2, "cluster": 3}
+
+
+def _assert_split(F, B, N, H, dh, rows, want, S_max=0, verify=False):
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("the shapes are chosen for 148 SMs")
+    mode, _ = F.fdllm_attention_split(B, N, H, dh, rows, S_max, verify)
+    assert mode == _SPLIT_CODE[want], f"attention split {mode}, expected {want}"
+
+
+@pytest.mark.parametrize("B,N,D,H,dh,nq,split", SPLIT_SHAPES)
+def test_attention_work_splits(F, B, N, D, H, dh, nq, split):
+    """Every way the attention spreads (sequence, head, chunk) items over the SMs
+    gives the oracle's result; the oracle checks up to four sequences (first,
+    last and two between), the cache outside Q is checked on all of them."""
+    _assert_split(F, B, N, H, dh, nq, split)
+    inp = W.random_fused(B, N, D, H, dh, nq=nq, seed=31 + B + N)
+    seqs = sorted({0, B // 3, (2 * B) // 3, B - 1})
+    _check_fused(F, inp, seqs_for_oracle=seqs)
+
+
+@pytest.mark.parametrize("B,N,D,H,dh,nq", [(12, 600, 128, 32, 64, 30), (3, 900, 128, 32, 128, 40)])
+def test_stream_k_deterministic(F, B, N, D, H, dh, nq):
+    """Stream-K merges a split item in CTA order by its last contributor: two
+    runs give the same bits whatever order the contributors finish in."""
+    _assert_split(F, B, N, H, dh, nq, "stream")
+    inp = W.random_fused(B, N, D, H, dh, nq=nq, seed=57)
+    a, b = W.to_device(inp), W.to_device(inp)
+    oa, _, sa = run_fused_gpu(F, a, 10000.0)
+    ob, _, sb = run_fused_gpu(F, b, 10000.0)
+    assert sa == F.OK and sb == F.OK
+    assert torch.equal(oa, ob)
+    assert torch.equal(a["k_cache"], b["k_cache"]) and torch.equal(a["v_cache"], b["v_cache"])
 
 
 @pytest.mark.parametrize("shape", [(1, 4096, 128, 1, 128, 20), (1, 6000, 128, 2, 64, 40)])
@@ -187,3 +239,35 @@ def test_stage_calls_equal_fused_call(F):
     F.fdllm_attend(q, b["k_cache"], b["v_cache"], out_s, ws)
     torch.cuda.synchronize()
     assert torch.equal(out_f, out_s) and torch.equal(a["k_cache"], b["k_cache"])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B,N,H,dh,nq", [(3, 400, 2, 128, 21), (16, 1024, 32, 128, 32)])
+def test_fused_step_rows_equals_fused_step(F, dtype, B, N, H, dh, nq):
+    """fdllm_fused_step_rows (x[Q] given packed) runs the same kernels on the same
+    rows as fdllm_fused_step: the same bits, caches included."""
+    inp = W.random_fused(B, N, 128, H, dh, nq=nq, dtype=dtype, seed=81 + B)
+    a, b = W.to_device(inp), W.to_device(inp)
+    out_f, _, st = run_fused_gpu(F, a, 10000.0)
+    assert st == F.OK
+    x_rows = torch.stack([b["x"][i, b["q_idx"][i].long()] for i in range(B)]).contiguous()
+    ws = F.alloc_workspace(F.fdllm_fused_step_workspace_bytes(B, N, 128, H, dh, nq, x_rows.dtype),
+                           "cuda")
+    out_r = torch.empty_like(out_f)
+    F.fdllm_fused_step_rows(x_rows, b["q_idx"], b["w_qkv"], b["k_cache"], b["v_cache"], out_r, ws)
+    assert F.fdllm_get_status(ws) == F.OK
+    assert torch.equal(out_f, out_r)
+    assert torch.equal(a["k_cache"], b["k_cache"]) and torch.equal(a["v_cache"], b["v_cache"])
+
+
+def test_fused_step_rows_reports_repeated_and_out_of_range_indices(F):
+    for q_idx in ([[3, 9, 3], [5, 6, 7]], [[3, 100, 7], [5, 6, 7]]):
+        inp = W.random_fused(2, 100, 128, 2, 64, q_idx=np.array([[3, 9, 4], [5, 6, 7]]), seed=11)
+        d = W.to_device(inp)
+        x_rows = torch.stack([d["x"][i, d["q_idx"][i].long()] for i in range(2)]).contiguous()
+        qi = torch.tensor(q_idx, dtype=torch.int32, device="cuda")
+        ws = F.alloc_workspace(F.fdllm_fused_step_workspace_bytes(2, 100, 128, 2, 64, 3,
+                                                                  torch.bfloat16), "cuda")
+        out = torch.empty((2, 3, 128), dtype=torch.bfloat16, device="cuda")
+        F.fdllm_fused_step_rows(x_rows, qi, d["w_qkv"], d["k_cache"], d["v_cache"], out, ws)
+        assert F.fdllm_get_status(ws) == F.ERR_BAD_INDEX

@@ -5,7 +5,8 @@ import torch
 
 import oracle as O
 import workloads as W
-from parity import assert_close, dtype_name, oracle_verify, run_verify_gpu
+from parity import (assert_close, check_outside_q_on_device, dtype_name, oracle_verify,
+                    run_verify_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -23,6 +24,20 @@ def _check_verify(F, inp, rope_base=10000.0, causal=False, seqs=None, inp_oracle
     k_in, v_in = inp["k_cache"].clone(), inp["v_cache"].clone()
     out, ws, st = run_verify_gpu(F, dev, rope_base, causal)
     assert st == F.OK, f"device status {st}"
+    # every sequence, sampled for the oracle or not: cache slots outside the
+    # T_v and draft positions, and side slots past the mask rows, bit-identical
+    pos_all, view_all = inp["pos"].numpy(), inp["view"].numpy()
+    Bn, Nn = inp["k_cache"].shape[0], inp["k_cache"].shape[2]
+    wmask = np.zeros((Bn, Nn), bool)
+    for b in range(Bn):
+        wmask[b, pos_all[b][(view_all[b] == 0) | (view_all[b] == 1)]] = True
+    check_outside_q_on_device(dev["k_cache"], inp["k_cache"], None, "k_cache", wmask)
+    check_outside_q_on_device(dev["v_cache"], inp["v_cache"], None, "v_cache", wmask)
+    for b in range(Bn):
+        n_side = int((view_all[b] == 2).sum())
+        for name in ("k_side", "v_side"):
+            assert torch.equal(dev[name][b][:, n_side:].cpu(), inp[name][b][:, n_side:]), \
+                f"{name}: an unused side slot changed in sequence {b}"
     dt = dtype_name(inp["x_rows"])
     H, dh = inp["k_cache"].shape[1], inp["k_cache"].shape[3]
     sel = list(range(inp["x_rows"].shape[0])) if seqs is None else list(seqs)
@@ -46,6 +61,52 @@ def _check_verify(F, inp, rope_base=10000.0, causal=False, seqs=None, inp_oracle
         assert_close(O.to_f64(vs[:, :n_side]), VS[i][:, :n_side], dt, "v side")
         assert torch.equal(ks[:, n_side:], inp["k_side"][sel[i]][:, n_side:])
     return out
+
+
+_SPLIT_CODE = {"stream": 1, "whole": 2, "cluster": 3}
+
+# (B, N, D, H, dh, |T_v|, |S|, split the attention must take on 148 SMs):
+# R = |T_v| + 2 |S| rows per sequence, query chunks of 16, 32 or 64 rows
+VERIFY_SPLITS = [
+    pytest.param(3, 700, 128, 32, 128, 4, 6, "stream", id="streamk-96items-nq16-dh128"),
+    pytest.param(3, 700, 128, 32, 128, 6, 12, "stream", id="streamk-96items-nq32-dh128"),
+    pytest.param(3, 700, 128, 32, 128, 8, 20, "stream", id="streamk-96items-nq64-dh128"),
+    pytest.param(3, 700, 128, 32, 64, 8, 20, "stream", id="streamk-96items-nq64-dh64"),
+    pytest.param(2, 700, 128, 32, 128, 20, 40, "stream", id="streamk-128items-2chunks-dh128"),
+    pytest.param(5, 1000, 128, 32, 128, 8, 16, "whole", id="whole-160items-nq64-dh128"),
+]
+
+
+def _assert_split(F, B, N, H, dh, R, S_max, want):
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("the shapes are chosen for 148 SMs")
+    mode, _ = F.fdllm_attention_split(B, N, H, dh, R, S_max, True)
+    assert mode == _SPLIT_CODE[want], f"attention split {mode}, expected {want}"
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["mutual", "causal"])
+@pytest.mark.parametrize("B,N,D,H,dh,n_tv,n_s,split", VERIFY_SPLITS)
+def test_verify_work_splits(F, B, N, D, H, dh, n_tv, n_s, split, causal):
+    """The view predicate under every work split of the attention, in both
+    visibility readings, against the oracle on every sequence."""
+    _assert_split(F, B, N, H, dh, n_tv + 2 * n_s, n_s, split)
+    inp = W.random_verify(B, N, D, H, dh, n_tv=n_tv, n_s=n_s, seed=61 + B + n_s)
+    _check_verify(F, inp, causal=causal)
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["mutual", "causal"])
+def test_verify_stream_k_deterministic(F, causal):
+    """Two stream-K verify passes on the same inputs give the same bits."""
+    B, N, D, H, dh, n_tv, n_s = 3, 700, 128, 32, 128, 8, 20
+    _assert_split(F, B, N, H, dh, n_tv + 2 * n_s, n_s, "stream")
+    inp = W.random_verify(B, N, D, H, dh, n_tv=n_tv, n_s=n_s, seed=67)
+    a, b = W.to_device(inp), W.to_device(inp)
+    oa, _, sa = run_verify_gpu(F, a, 10000.0, causal)
+    ob, _, sb = run_verify_gpu(F, b, 10000.0, causal)
+    assert sa == F.OK and sb == F.OK
+    assert torch.equal(oa, ob)
+    for k in ("k_cache", "v_cache", "k_side", "v_side"):
+        assert torch.equal(a[k], b[k]), k
 
 
 def test_verify_bf16_config_sampled(F):

@@ -2,16 +2,19 @@
 device memory where they call the library (a plugin handed only its buffers, a
 runtime whose memory is all reserved, a loop where cudaMalloc would stall).
 
-It must give what fdllm_accept gives on the same inputs, on two calls in a row
-(the second call reuses the library's fixed scratch array, which still holds the
-first call's contents).  This file sorts last so that a run stopping at the
-first failure has already run every other test."""
+It runs the same kernel as fdllm_accept, with the same split of each row, so
+it must give the same bits on the same inputs, on two calls in a row (the
+second call reuses the library's fixed scratch array, which still holds the
+first call's partials).  A clean call leaves the array's counters at zero
+itself; the call's own clearing of them guards only against an earlier launch
+that was cut short, which these two calls do not exercise.  This file sorts
+last so that a run stopping at the first failure has already run every other
+test."""
 import numpy as np
 import pytest
 import torch
 
 import workloads as W
-from parity import CONF_TOL
 
 pytestmark = pytest.mark.gpu
 
@@ -32,7 +35,7 @@ def _compare(F, logits, kind, ref_tok, rank, eps, gamma):
     F.fdllm_accept_noalloc(logits, kind, ref_tok, rank, *got, eps=eps, gamma=gamma)
     torch.cuda.synchronize()
     assert torch.equal(got[0], ref[0])                                   # top1
-    assert (got[1] - ref[1]).abs().max().item() <= CONF_TOL              # conf
+    assert torch.equal(got[1], ref[1])                                   # conf, bit for bit
     assert torch.equal(got[2], ref[2]) and torch.equal(got[3], ref[3])   # flags, n_accept
 
 
