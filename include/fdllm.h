@@ -210,10 +210,11 @@ fdllm_status fdllm_accept(int B, int R, int V, const float* logits, const int8_t
  *   minus the workspace.  The call allocates nothing (no cudaMalloc, no
  *   cudaFree, no allocating library routine).  Its scratch is a device array of
  *   FDLLM_ACCEPT_NOALLOC_SCRATCH_BYTES compiled into the library: every GPU that
- *   loads the library holds it until the process exits.  It needs
- *   align256(B*R*splits*16) + align256(B*R*4) + align256(B*4) bytes, where
- *   splits <= max(1, 8*SMs / (B*R)); B*R <= 131072 always fits, and a call that
- *   does not fit returns FDLLM_ERR_UNSUPPORTED without launching anything.
+ *   loads the library holds it until the process exits.  A call needs at most
+ *   align256(16*(B*R + 8*SMs)) + align256(4*B*R) + align256(4*B) bytes of it
+ *   (the row partials of the scan, then per-row and per-sequence counters);
+ *   B*R <= 131072 always fits on GPUs of up to 256 SMs, and a call that does not
+ *   fit returns FDLLM_ERR_UNSUPPORTED without launching anything.
  *   Every call on a device shares the one array, which keeps the last call's
  *   contents; each call first clears (cudaMemsetAsync on `stream`) the counters
  *   that must start at zero.  Calls that overlap on the GPU (on different

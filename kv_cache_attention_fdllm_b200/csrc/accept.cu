@@ -55,7 +55,7 @@ __device__ __forceinline__ void fold1(MaxSum& s, float x, int i) {
     s.l = s.l * scale_to(s.m, x) + 1.f;
     s.m = x;
     s.idx = i;
-  } else {
+  } else if (x > -INFINITY) {  // a -inf logit adds nothing (and s.m is finite here)
     s.l += exp2f((x - s.m) * kLog2e);
   }
 }
@@ -112,14 +112,16 @@ accept_kernel(int R, int V, int splits, int span, const float* __restrict__ logi
       st.m = cm;
       st.idx = ci;
     }
-    const float ms = st.m * kLog2e;
-    float acc = 0.f;
+    if (st.m > -INFINITY) {  // else this thread has seen nothing but -inf so far
+      const float ms = st.m * kLog2e;
+      float acc = 0.f;
 #pragma unroll
-    for (int u = 0; u < kAcceptUnroll; ++u) {
-      acc += exp2f(fmaf(v[u].x, kLog2e, -ms)) + exp2f(fmaf(v[u].y, kLog2e, -ms)) +
-             exp2f(fmaf(v[u].z, kLog2e, -ms)) + exp2f(fmaf(v[u].w, kLog2e, -ms));
+      for (int u = 0; u < kAcceptUnroll; ++u) {
+        acc += exp2f(fmaf(v[u].x, kLog2e, -ms)) + exp2f(fmaf(v[u].y, kLog2e, -ms)) +
+               exp2f(fmaf(v[u].z, kLog2e, -ms)) + exp2f(fmaf(v[u].w, kLog2e, -ms));
+      }
+      st.l += acc;
     }
-    st.l += acc;
   }
   if (a1 + tid < s1) fold1(st, p[a1 + tid], a1 + tid);
 
@@ -213,25 +215,31 @@ accept_kernel(int R, int V, int splits, int span, const float* __restrict__ logi
 
 }  // namespace
 
-int accept_splits(int rows, int V, int num_sms) {
+AcceptLayout accept_layout(int B, int R, int V, int num_sms) {
+  AcceptLayout L{};
+  const long long rows = (long long)B * R;
   // one wave of resident CTAs (8 per SM at 256 threads), at least 2048
   // elements per CTA, at most one split per row when the rows fill the GPU
   const int resident = num_sms * 8;
-  int s = resident / (rows > 0 ? rows : 1);
+  int sp = (int)(resident / (rows > 0 ? rows : 1));
   const int max_s = (V + 2047) / 2048;
-  if (s > max_s) s = max_s;
-  if (s < 1) s = 1;
-  return s;
+  if (sp > max_s) sp = max_s;
+  if (sp < 1) sp = 1;
+  L.splits = sp;
+  L.parts_bytes = align_up((size_t)rows * sp * sizeof(AcceptPartial), 256);
+  L.row_cnt_bytes = align_up((size_t)rows * sizeof(unsigned), 256);
+  L.seq_cnt_bytes = align_up((size_t)(B > 0 ? B : 1) * sizeof(unsigned), 256);
+  return L;
 }
 
-cudaError_t launch_accept(const AcceptArgs& a, cudaStream_t stream) {
+cudaError_t launch_accept(const AcceptArgs& a, const AcceptLayout& L, cudaStream_t stream) {
   const int rows = a.B * a.R;
   if (rows == 0) return cudaSuccess;
-  int span = (a.V + a.splits - 1) / a.splits;
+  int span = (a.V + L.splits - 1) / L.splits;
   span = (span + 3) & ~3;
-  dim3 grid(rows, a.splits);
+  dim3 grid(rows, L.splits);
   accept_kernel<<<grid, kAcceptThreads, 0, stream>>>(
-      a.R, a.V, a.splits, span, a.logits, a.kind, a.ref_tok, a.rank, a.eps, a.gamma, a.top1,
+      a.R, a.V, L.splits, span, a.logits, a.kind, a.ref_tok, a.rank, a.eps, a.gamma, a.top1,
       a.conf, a.flags, a.n_accept, a.parts, a.row_cnt, a.seq_cnt);
   count_launches(1);
   return cudaGetLastError();

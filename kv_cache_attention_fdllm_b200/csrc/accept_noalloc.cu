@@ -104,12 +104,9 @@ extern "C" fdllm_status fdllm_accept_noalloc(int B, int R, int V, const float* l
   if ((long long)B * R > (1ll << 31) - 1 || (long long)B * R * V > (1ll << 40))
     return FDLLM_ERR_UNSUPPORTED;
   const int rows = B * R;
-  const int splits = accept_splits(rows, V, device_sm_count());
+  const AcceptLayout AL = accept_layout(B, R, V, device_sm_count());
   // scratch layout: [partials | per-row counters | per-sequence counters]
-  const size_t parts_bytes = align_up((size_t)rows * splits * sizeof(AcceptPartial), 256);
-  const size_t row_cnt_bytes = align_up((size_t)rows * sizeof(unsigned), 256);
-  const size_t seq_cnt_bytes = align_up((size_t)(B > 0 ? B : 1) * sizeof(unsigned), 256);
-  if (parts_bytes + row_cnt_bytes + seq_cnt_bytes > kScratchBytes) return FDLLM_ERR_UNSUPPORTED;
+  if (AL.total() > kScratchBytes) return FDLLM_ERR_UNSUPPORTED;
   if (rows == 0) return FDLLM_OK;
   if (!logits || !kind || !top1 || !conf || !flags || !n_accept) return FDLLM_ERR_INVALID_ARG;
   if (!is_aligned16(logits) || !is_aligned16(kind) || !is_aligned16(top1) ||
@@ -124,16 +121,17 @@ extern "C" fdllm_status fdllm_accept_noalloc(int B, int R, int V, const float* l
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* p = static_cast<char*>(base);
   // the counters must start at zero; the array keeps whatever the last call left
-  if (cudaMemsetAsync(p + parts_bytes, 0, row_cnt_bytes + seq_cnt_bytes, s) != cudaSuccess)
+  if (cudaMemsetAsync(p + AL.parts_bytes, 0, AL.row_cnt_bytes + AL.seq_cnt_bytes,
+                      s) != cudaSuccess)
     return FDLLM_ERR_CUDA;
 
   AcceptArgs a{};
-  a.B = B; a.R = R; a.V = V; a.splits = splits;
+  a.B = B; a.R = R; a.V = V;
   a.logits = logits; a.kind = kind; a.ref_tok = ref_tok; a.rank = rank;
   a.eps = eps; a.gamma = gamma;
   a.top1 = top1; a.conf = conf; a.flags = flags; a.n_accept = n_accept;
   a.parts = reinterpret_cast<AcceptPartial*>(p);
-  a.row_cnt = reinterpret_cast<unsigned*>(p + parts_bytes);
-  a.seq_cnt = reinterpret_cast<unsigned*>(p + parts_bytes + row_cnt_bytes);
-  return launch_accept(a, s) == cudaSuccess ? FDLLM_OK : FDLLM_ERR_CUDA;
+  a.row_cnt = reinterpret_cast<unsigned*>(p + AL.parts_bytes);
+  a.seq_cnt = reinterpret_cast<unsigned*>(p + AL.parts_bytes + AL.row_cnt_bytes);
+  return launch_accept(a, AL, s) == cudaSuccess ? FDLLM_OK : FDLLM_ERR_CUDA;
 }

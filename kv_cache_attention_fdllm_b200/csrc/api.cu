@@ -174,13 +174,7 @@ size_t fdllm_verify_step_workspace_bytes(int B, int N, int D, int H, int dh, int
 
 size_t fdllm_accept_workspace_bytes(int B, int R, int V) {
   if (B < 0 || R < 0 || V < 1) return 0;
-  const int rows = B * R;
-  const int splits = accept_splits(rows, V, device_sm_count());
-  size_t off = kWsHeaderBytes;
-  off += align_up((size_t)rows * splits * sizeof(AcceptPartial), 256);
-  off += align_up((size_t)rows * sizeof(unsigned), 256);
-  off += align_up((size_t)(B > 0 ? B : 1) * sizeof(unsigned), 256);
-  return off;
+  return kWsHeaderBytes + accept_layout(B, R, V, device_sm_count()).total();
 }
 
 fdllm_status fdllm_qkv_rope_scatter(int B, int N, int D, int H, int dh, int nq, int dtype,
@@ -343,20 +337,19 @@ fdllm_status fdllm_accept(int B, int R, int V, const float* logits, const int8_t
   if ((ref_tok && !aligned16(ref_tok)) || (rank && !aligned16(rank)))
     return FDLLM_ERR_INVALID_ARG;
   // kind-2 rows need ref_tok and rank; the kernel reads them only for such rows
-  const int rows = B * R;
+  const AcceptLayout AL = accept_layout(B, R, V, device_sm_count());
   AcceptArgs a{};
   a.B = B; a.R = R; a.V = V;
-  a.splits = accept_splits(rows, V, device_sm_count());
   a.logits = logits; a.kind = kind; a.ref_tok = ref_tok; a.rank = rank;
   a.eps = eps; a.gamma = gamma;
   a.top1 = top1; a.conf = conf; a.flags = flags; a.n_accept = n_accept;
   size_t off = kWsHeaderBytes;
   a.parts = reinterpret_cast<AcceptPartial*>(ws_at(workspace, off));
-  off += align_up((size_t)rows * a.splits * sizeof(AcceptPartial), 256);
+  off += AL.parts_bytes;
   a.row_cnt = reinterpret_cast<unsigned*>(ws_at(workspace, off));
-  off += align_up((size_t)rows * sizeof(unsigned), 256);
+  off += AL.row_cnt_bytes;
   a.seq_cnt = reinterpret_cast<unsigned*>(ws_at(workspace, off));
-  return from_cuda(launch_accept(a, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_accept(a, AL, static_cast<cudaStream_t>(stream)));
 }
 
 fdllm_status fdllm_track_select(int B, int N, int H, int dh, int nq, int dtype,

@@ -53,6 +53,7 @@ constexpr int kKT = 128;  // keys per tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kThresh = 8.f;  // lazy rescale threshold (log2 units)
 constexpr int kMaxRows = 512;   // verify rows per sequence held in shared memory
+constexpr int kDraftTab = 2048; // cache slots a segment's draft-rank table covers
 constexpr int kL2PrefetchTiles = 4;  // cache tiles per CTA warmed in L2 before the dependency wait
 // work splits (the values fdllm_attention_split reports)
 constexpr int kSplitStreamK = 1, kSplitWholeItems = 2, kSplitClusters = 3;
@@ -231,6 +232,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   int* draft_pos = reinterpret_cast<int*>(misc + 4096);     // [kMaxRows]
   int* draft_rank = draft_pos + kMaxRows;                   // [kMaxRows]
   int* side_rank = draft_rank + kMaxRows;                   // [kMaxRows]
+  // draft rank of each cache slot in [d_lo, d_lo + kDraftTab), -1 for no draft
+  int16_t* kdr_tab = reinterpret_cast<int16_t*>(side_rank + kMaxRows);  // [kDraftTab]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -457,6 +460,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float l[NQH], mrun[NQH];
     int seg = -1;
     int n_draft = 0, n_side = 0, d_lo = INT_MAX, d_hi = INT_MIN;
+    bool tab = false;      // the segment's draft positions are in kdr_tab
+    uint32_t v2cols = 0;   // bit c: this thread's column c0 + c is a mask-view row
     int pv_waited = -1;  // index of the last PV this thread waited for
     int seg_t0 = 0;      // tile index at which the current segment started
     UnitCursor cs;
@@ -522,6 +527,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           n_side = *n_side_s;
           d_lo = *d_lo_s;
           d_hi = *d_hi_s;
+          // slot -> draft rank, one shared-memory load per key instead of a scan
+          // of the drafts, when their positions span at most kDraftTab slots
+          tab = n_draft > 0 && d_hi - d_lo < kDraftTab;
+          if (tab) {
+            for (int j = st; j <= d_hi - d_lo; j += kSmx) kdr_tab[j] = -1;
+            tc::named_bar_sync(1, kSmx);
+            for (int d = st; d < n_draft; d += kSmx) kdr_tab[draft_pos[d] - d_lo] = (int16_t)draft_rank[d];
+            tc::named_bar_sync(1, kSmx);
+          }
+          v2cols = 0;
+#pragma unroll
+          for (int c = 0; c < NQH; ++c)
+            if ((col_meta[c0 + c] & 3) == 2) v2cols |= 1u << c;
         }
       }
 
@@ -545,25 +563,44 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
         for (int c = 0; c < NQH; ++c) s[c] = -INFINITY;
       } else if (VERIFY) {
+        // The view rule (visible_side / visible_cache).  In the mutual reading
+        // it depends only on whether the column is a mask-view row, a bit of
+        // v2cols; the causal reading also compares ranks.
         if (side_tile) {
-          const int srank = side_rank[key];
+          if (!p.causal) {
 #pragma unroll
-          for (int c = 0; c < NQH; ++c) {
-            const int cm = col_meta[c0 + c];
-            if (!visible_side(cm & 3, cm >> 2, srank, p.causal)) s[c] = -INFINITY;
-          }
-        } else {
-          // only tiles that reach the draft positions' range need the lookup
-          int kdr = -1;
-          const int tk0 = t * kKT;
-          if (tk0 <= d_hi && tk0 + kKT > d_lo)
-            for (int d = 0; d < n_draft; ++d)
-              if (draft_pos[d] == key) kdr = draft_rank[d];
-          if (kdr >= 0) {
+            for (int c = 0; c < NQH; ++c)
+              if (!((v2cols >> c) & 1u)) s[c] = -INFINITY;
+          } else {
+            const int srank = side_rank[key];
 #pragma unroll
             for (int c = 0; c < NQH; ++c) {
               const int cm = col_meta[c0 + c];
-              if (!visible_cache(cm & 3, cm >> 2, kdr, p.causal)) s[c] = -INFINITY;
+              if (!visible_side(cm & 3, cm >> 2, srank, 1)) s[c] = -INFINITY;
+            }
+          }
+        } else {
+          // only keys within the draft positions' range need the lookup
+          int kdr = -1;
+          if (key >= d_lo && key <= d_hi) {
+            if (tab) {
+              kdr = kdr_tab[key - d_lo];
+            } else {
+              for (int d = 0; d < n_draft; ++d)
+                if (draft_pos[d] == key) kdr = draft_rank[d];
+            }
+          }
+          if (kdr >= 0) {
+            if (!p.causal) {
+#pragma unroll
+              for (int c = 0; c < NQH; ++c)
+                if ((v2cols >> c) & 1u) s[c] = -INFINITY;
+            } else {
+#pragma unroll
+              for (int c = 0; c < NQH; ++c) {
+                const int cm = col_meta[c0 + c];
+                if (!visible_cache(cm & 3, cm >> 2, kdr, 1)) s[c] = -INFINITY;
+              }
             }
           }
         }
@@ -965,7 +1002,7 @@ AttnPlan plan(int B, int N, int H, int dh, int rows, int S_max, int verify, int 
   const size_t pbytes = 2 * (((size_t)kKT * q.NQ * 2 + 1023) / 1024 * 1024);
   // misc: barriers and softmax scratch, then the verify tables (or, without
   // them, the [8][NQ] merge weights of the stream-K path)
-  const size_t misc = 4096 + (verify ? 3 * kMaxRows * 4 : 8 * 64 * 4);
+  const size_t misc = 4096 + (verify ? 3 * kMaxRows * 4 + kDraftTab * 2 : 8 * 64 * 4);
   // K and V tiles share what shared memory is left.  A V tile is held from its
   // load until its PV is done, longer than a K tile, so V gets the odd one.
   // Cluster mode runs one item per CTA and needs one Q buffer, not two.

@@ -16,7 +16,7 @@ struct AcceptPartial {
 };
 
 struct AcceptArgs {
-  int B, R, V, splits;
+  int B, R, V;
   const float* logits;
   const int8_t* kind;
   const int32_t* ref_tok;
@@ -26,13 +26,20 @@ struct AcceptArgs {
   float* conf;
   uint8_t* flags;
   int32_t* n_accept;
-  AcceptPartial* parts;  // [B*R*splits]
+  AcceptPartial* parts;  // layout.parts_bytes
   unsigned* row_cnt;     // [B*R], zero between calls
   unsigned* seq_cnt;     // [B], zero between calls
 };
 
-int accept_splits(int rows, int V, int num_sms);
-cudaError_t launch_accept(const AcceptArgs& a, cudaStream_t stream);
+// How the acceptance scan is split (grid rows x splits, each CTA one span of
+// one row), and the scratch it needs.
+struct AcceptLayout {
+  int splits;
+  size_t parts_bytes, row_cnt_bytes, seq_cnt_bytes;
+  size_t total() const { return parts_bytes + row_cnt_bytes + seq_cnt_bytes; }
+};
+AcceptLayout accept_layout(int B, int R, int V, int num_sms);
+cudaError_t launch_accept(const AcceptArgs& a, const AcceptLayout& L, cudaStream_t stream);
 
 // ----------------------------------------------------------------- projection
 // Rows of the projection: token m of sequence b = m / rows_per_seq.

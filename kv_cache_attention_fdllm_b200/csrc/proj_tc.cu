@@ -18,7 +18,10 @@
 //
 // Persistent stream-K: one CTA per SM.  The (tile, k-step) units are laid out
 // tile after tile and every CTA takes an equal contiguous range of them, so the
-// load is balanced whatever the tile count.  A CTA's range covers whole tiles
+// load is balanced whatever the tile count.  Tiles are numbered feature tile
+// first (tile = token tile * feature tiles + feature tile): the CTAs that work
+// on the token tiles of one feature tile then run side by side, so W streams
+// from HBM once and the other token tiles find it in L2.  A CTA's range covers whole tiles
 // and at most one partial tile at each end; a partial tile is written as an
 // fp32 partial and the last of its contributors (atomic counter) sums the
 // partials in k order (results do not depend on timing) and runs the epilogue.
@@ -57,7 +60,7 @@ constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
 struct ProjTcParams {
   int M, F, D, E, N, H, dh, rows_per_seq, S_max, verify;
   int check_repeats;   // report a repeated index (packed fused rows; the prep kernel does it otherwise)
-  int BN, n_tt, tiles, nks, subs, nsub_total, nstage;
+  int BN, n_tt, n_ft, tiles, nks, subs, nsub_total, nstage;
   long long total_units;
   const int32_t* idx;
   const int8_t* view;
@@ -200,7 +203,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         tc::mbar_arrive_expect_tx(&full[i], (uint32_t)nsub * (kASubBytes + bsub_bytes));
         for (int q = 0; q < nsub; ++q)
           tc::tma_load_2d(a_s + q * kASubBytes, &tm_w, &full[i], (sb0 + q) * kSub,
-                          (tile / p.n_tt) * kBM, pol_w);
+                          (tile % p.n_ft) * kBM, pol_w);
       }
       tc::griddep_wait();
       tile = tile_begin;
@@ -214,7 +217,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         uint8_t* b_s = smem + i * stage_bytes + p.subs * kASubBytes;
         for (int q = 0; q < nsub; ++q)
           tc::tma_load_2d(b_s + q * bsub_bytes, &tm_x, &full[i], (sb0 + q) * kSub,
-                          (tile % p.n_tt) * BN, pol_x);
+                          (tile / p.n_ft) * BN, pol_x);
       }
       for (int it = pre; it < (int)n_units; ++it) {
         if (++ks == p.nks) {
@@ -231,9 +234,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         tc::mbar_arrive_expect_tx(&full[s], (uint32_t)nsub * (kASubBytes + bsub_bytes));
         for (int q = 0; q < nsub; ++q) {
           tc::tma_load_2d(a_s + q * kASubBytes, &tm_w, &full[s], (sb0 + q) * kSub,
-                          (tile / p.n_tt) * kBM, pol_w);
+                          (tile % p.n_ft) * kBM, pol_w);
           tc::tma_load_2d(b_s + q * bsub_bytes, &tm_x, &full[s], (sb0 + q) * kSub,
-                          (tile % p.n_tt) * BN, pol_x);
+                          (tile / p.n_ft) * BN, pol_x);
         }
       }
     }
@@ -297,7 +300,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       const int ks1 = (int)min((long long)p.nks, ks0 + (u_end - u));
       u += ks1 - ks0;
       const int buf = j & 1;
-      const int ft = tile / p.n_tt, tt = tile % p.n_tt;
+      const int ft = tile % p.n_ft, tt = tile / p.n_ft;
       const int m0 = tt * BN;
       const bool whole = (ks0 == 0 && ks1 == p.nks);
       const uint32_t t_acc = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
@@ -587,7 +590,7 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream) {
   p.M = M; p.F = F; p.D = a.D; p.E = E; p.N = a.N; p.H = a.H; p.dh = a.dh;
   p.rows_per_seq = a.rows_per_seq; p.S_max = a.S_max; p.verify = a.verify;
   p.check_repeats = (!a.verify && a.packed) ? 1 : 0;
-  p.BN = q.BN; p.n_tt = q.n_tt; p.tiles = q.tiles; p.nks = q.nks; p.subs = q.subs;
+  p.BN = q.BN; p.n_tt = q.n_tt; p.n_ft = q.n_ft; p.tiles = q.tiles; p.nks = q.nks; p.subs = q.subs;
   p.nsub_total = q.nsub_total; p.nstage = q.nstage; p.total_units = q.total_units;
   p.idx = a.idx; p.view = a.view; p.log2_base = a.log2_base;
   p.k_cache = static_cast<__nv_bfloat16*>(a.k_cache);

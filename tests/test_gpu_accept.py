@@ -122,3 +122,51 @@ def test_repeated_calls_reuse_workspace(F):
         res.append((top1.clone(), conf.clone(), flags.clone(), n.clone()))
     for r in res[1:]:
         assert all(torch.equal(x, y) for x, y in zip(r, res[0]))
+
+
+@pytest.mark.parametrize("B,R,V", [(2, 160, 4096), (3, 7, 60001), (1, 25, 126464), (4, 80, 9000)])
+def test_long_rows_split_over_ctas(F, B, R, V):
+    """Rows split over several CTAs, many rows per sequence, and a vocabulary
+    that is not a multiple of four (rows start off 16-byte boundaries)."""
+    logits, tok = W.random_logits(B, R, V, seed=B * R + V)
+    g = np.random.default_rng(V)
+    kind = torch.from_numpy(g.integers(0, 3, (B, R)).astype(np.int8))
+    ref = torch.from_numpy(np.where(g.random((B, R)) < 0.7, tok, (tok + 1) % V).astype(np.int32))
+    rank = torch.from_numpy(np.stack([g.permutation(R) for _ in range(B)]).astype(np.int32))
+    gpu, refr = _run_both(F, logits.cuda(), kind, ref, rank, 0.6, 0.5)
+    check_accept(gpu, refr, kind.numpy(), rank.numpy(), 0.6, 0.5)
+
+
+def test_ties_across_splits_and_masked_logits(F):
+    """The largest logit tied at two places of a row that different CTAs hold
+    (the lower index wins), the maximum in a row's last element, and -inf
+    logits (a masked vocabulary entry adds nothing to the sum)."""
+    B, R, V = 1, 40, 126464
+    g = torch.Generator().manual_seed(9)
+    l = torch.randn((B, R, V), generator=g)
+    l[0, 0, 5] = 9.0
+    l[0, 0, V - 7] = 9.0                   # same value far apart: index 5 wins
+    l[0, 1, V - 1] = 12.0                  # the maximum in the last element
+    l[0, 2, ::3] = -float("inf")           # a third of the row masked out
+    l[0, 3, :] = -float("inf")
+    l[0, 3, 77] = 0.0                      # one finite logit: confidence 1
+    kind = torch.ones((B, R), dtype=torch.int8)
+    gpu, ref = _run_both(F, l.cuda(), kind, torch.zeros((B, R), dtype=torch.int32),
+                         torch.zeros((B, R), dtype=torch.int32), 0.9, 0.8)
+    assert gpu[0][0, 0] == 5 and gpu[0][0, 1] == V - 1 and gpu[0][0, 3] == 77
+    assert gpu[1][0, 3] == 1.0
+    assert np.isfinite(gpu[1]).all()
+    check_accept(gpu, ref, kind.numpy(), np.zeros((B, R), np.int64), 0.9, 0.8)
+
+
+def test_long_rows_deterministic(F):
+    B, R, V = 8, 40, 126464
+    logits, tok = W.random_logits(B, R, V, seed=17)
+    kind = torch.full((B, R), 2, dtype=torch.int8).cuda()
+    rank = torch.arange(R, dtype=torch.int32).repeat(B, 1).cuda()
+    ref_tok = torch.from_numpy(tok).cuda()
+    d = logits.cuda()
+    a = run_accept_gpu(F, d, kind, ref_tok, rank, 0.9, 0.8)[:4]
+    b = run_accept_gpu(F, d, kind, ref_tok, rank, 0.9, 0.8)[:4]
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
