@@ -171,13 +171,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Columns a query chunk occupies in TMEM and in P's swizzled layout: 48
+// queries run the MMAs with N = 48 but keep the 64-column layout (P rows of
+// 128 bytes, one 128-byte swizzle atom; TMEM buffers 64 columns apart).
+template <int NQ>
+struct NQP {
+  static constexpr int v = NQ == 48 ? 64 : NQ;
+};
+
 // Shared-memory layout of one CTA (offsets from a 1024-aligned base).
 template <int NQ, int DH>
 struct Smem {
   static constexpr int kBoxes = DH / 64;
   static constexpr uint32_t kTileBytes = kBoxes * 16384;         // K or V tile
   static constexpr uint32_t kQBytes = kBoxes * NQ * 128;         // one Q chunk
-  static constexpr uint32_t kPRow = NQ * 2;                      // bytes per key row of P
+  static constexpr uint32_t kPRow = NQP<NQ>::v * 2;              // bytes per key row of P
   static constexpr uint32_t kPBytes = kKT * kPRow;
   static constexpr uint32_t kPBufBytes = (kPBytes + 1023) / 1024 * 1024;  // one of two P buffers
 };
@@ -255,7 +263,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int T = (int)(u1 - u0);
 
   uint32_t ncols = 32;
-  while ((int)ncols < 3 * NQ) ncols <<= 1;
+  while ((int)ncols < 3 * NQP<NQ>::v) ncols <<= 1;
 
   if (tid == 0) {
     for (int s = 0; s < NK; ++s) {
@@ -304,7 +312,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_o = tmem + 2 * NQ;
+  const uint32_t tmem_o = tmem + 2 * NQP<NQ>::v;
   // every thread: nothing written by an earlier kernel is read before this
   tc::griddep_wait();
 
@@ -380,7 +388,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (lane == 0) {
       constexpr uint32_t idesc_qk = tc::idesc_bf16(kKT, NQ, false, false);
       constexpr uint32_t idesc_pv = tc::idesc_bf16(kKT, NQ, true, true);
-      constexpr uint32_t p_swz = NQ == 64 ? 2u : (NQ == 32 ? 4u : 6u);
+      constexpr uint32_t p_swz = L::kPRow == 128 ? 2u : (L::kPRow == 64 ? 4u : 6u);
       const uint32_t p_addr = tc::smem_u32(p_buf);
       int iq = 0, ip = 0, seg = -1;
       UnitCursor cq, cpv;
@@ -407,7 +415,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int kk = 0; kk < DH / 16; ++kk) {
               const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
               const uint32_t qo = (kk >> 2) * NQ * 128 + (kk & 3) * 32;
-              tc::mma_bf16(tmem + sb * NQ, tc::smem_desc(k_addr + ko, 16, 1024, 2),
+              tc::mma_bf16(tmem + sb * NQP<NQ>::v, tc::smem_desc(k_addr + ko, 16, 1024, 2),
                            tc::smem_desc(q_addr + qo, 16, 1024, 2), idesc_qk, kk != 0);
             }
             tc::mma_commit(&s_full[sb]);
@@ -550,7 +558,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc::mbar_wait(&s_full[sb], (uint32_t)(i >> 1) & 1u, abort_flag, p.status);
       tc::tc_fence_after();
       float s[NQH];
-      tmem_ld_row<NQH>(tmem + lane_off + sb * NQ + c0, s);
+      tmem_ld_row<NQH>(tmem + lane_off + sb * NQP<NQ>::v + c0, s);
       tc::tmem_wait_ld();
       tc::tc_fence_before();
       __syncwarp();
@@ -888,7 +896,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             if (st < NQ && p.lse && qc * NQ + st < p.rows)
               p.lse[((size_t)b * p.rows + qc * NQ + st) * p.H + h] = M + log2f(Lsum);
-            constexpr int kJ = NQ == 64 ? 2 : 4;  // contributors per batch of O loads
+            constexpr int kJ = NQH == 32 ? 2 : 4;  // contributors per batch of O loads
             float acc[NQH];
 #pragma unroll
             for (int c = 0; c < NQH; ++c) acc[c] = 0.f;
@@ -980,7 +988,7 @@ constexpr size_t kSmemBudget = 227 * 1024;
 
 AttnPlan plan(int B, int N, int H, int dh, int rows, int S_max, int verify, int num_sms) {
   AttnPlan q{};
-  q.NQ = rows <= 16 ? 16 : (rows <= 32 ? 32 : 64);
+  q.NQ = rows <= 16 ? 16 : (rows <= 32 ? 32 : (rows <= 48 ? 48 : 64));
   q.n_qc = (rows + q.NQ - 1) / q.NQ;
   q.nct = (N + kKT - 1) / kKT;
   q.nst = (verify && S_max > 0) ? (S_max + kKT - 1) / kKT : 0;
@@ -999,7 +1007,8 @@ AttnPlan plan(int B, int N, int H, int dh, int rows, int S_max, int verify, int 
   const size_t boxes = dh / 64;
   const size_t tile = boxes * 16384;
   const size_t qbytes = boxes * q.NQ * 128;
-  const size_t pbytes = 2 * (((size_t)kKT * q.NQ * 2 + 1023) / 1024 * 1024);
+  const size_t nqp = q.NQ == 48 ? 64 : q.NQ;  // P's padded columns
+  const size_t pbytes = 2 * (((size_t)kKT * nqp * 2 + 1023) / 1024 * 1024);
   // misc: barriers and softmax scratch, then the verify tables (or, without
   // them, the [8][NQ] merge weights of the stream-K path)
   const size_t misc = 4096 + (verify ? 3 * kMaxRows * 4 + kDraftTab * 2 : 8 * 64 * 4);
@@ -1152,9 +1161,11 @@ int attn_tc_split(int B, int N, int H, int dh, int rows, int S_max, int verify, 
                : resolve_split<NQv, DHv, false>(q, &mode, cs);
   FDLLM_ATTN_SPLIT(16, 64)
   FDLLM_ATTN_SPLIT(32, 64)
+  FDLLM_ATTN_SPLIT(48, 64)
   FDLLM_ATTN_SPLIT(64, 64)
   FDLLM_ATTN_SPLIT(16, 128)
   FDLLM_ATTN_SPLIT(32, 128)
+  FDLLM_ATTN_SPLIT(48, 128)
   FDLLM_ATTN_SPLIT(64, 128)
 #undef FDLLM_ATTN_SPLIT
   return e == cudaSuccess ? mode : -1;
@@ -1212,9 +1223,11 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
                     : launch_t<NQv, DHv, false>(a, q, prm, maps, stream);
   FDLLM_ATTN_CASE(16, 64)
   FDLLM_ATTN_CASE(32, 64)
+  FDLLM_ATTN_CASE(48, 64)
   FDLLM_ATTN_CASE(64, 64)
   FDLLM_ATTN_CASE(16, 128)
   FDLLM_ATTN_CASE(32, 128)
+  FDLLM_ATTN_CASE(48, 128)
   FDLLM_ATTN_CASE(64, 128)
 #undef FDLLM_ATTN_CASE
   return cudaErrorInvalidValue;

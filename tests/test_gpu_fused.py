@@ -86,7 +86,9 @@ SPLIT_SHAPES = [
     pytest.param(5, 1000, 128, 32, 64, 20, "whole", id="whole-160items-nq32-dh64"),
     pytest.param(12, 700, 128, 16, 128, 12, "whole", id="whole-192items-nq16-dh128"),
     pytest.param(8, 1024, 128, 32, 128, 32, "whole", id="whole-256items-nq32-dh128"),
-    pytest.param(3, 900, 128, 32, 128, 40, "stream", id="streamk-96items-nq64-dh128"),
+    pytest.param(5, 1000, 128, 32, 128, 40, "whole", id="whole-160items-nq48-dh128"),
+    pytest.param(3, 900, 128, 32, 128, 60, "stream", id="streamk-96items-nq64-dh128"),
+    pytest.param(3, 900, 128, 32, 64, 44, "stream", id="streamk-96items-nq48-dh64"),
     pytest.param(12, 600, 128, 32, 64, 30, "stream", id="streamk-384items-nq32-dh64"),
     pytest.param(2, 800, 128, 32, 64, 100, "stream", id="streamk-128items-2chunks-dh64"),
     pytest.param(16, 1024, 128, 32, 128, 32, "stream", id="streamk-512items-nq32-dh128"),
@@ -112,7 +114,8 @@ def test_attention_work_splits(F, B, N, D, H, dh, nq, split):
     _check_fused(F, inp, seqs_for_oracle=seqs)
 
 
-@pytest.mark.parametrize("B,N,D,H,dh,nq", [(12, 600, 128, 32, 64, 30), (3, 900, 128, 32, 128, 40)])
+@pytest.mark.parametrize("B,N,D,H,dh,nq", [(12, 600, 128, 32, 64, 30), (3, 900, 128, 32, 128, 40),
+                                            (3, 900, 128, 32, 128, 60)])
 def test_stream_k_deterministic(F, B, N, D, H, dh, nq):
     """Stream-K merges a split item in CTA order by its last contributor: two
     runs give the same bits whatever order the contributors finish in."""

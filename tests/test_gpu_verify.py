@@ -70,10 +70,12 @@ _SPLIT_CODE = {"stream": 1, "whole": 2, "cluster": 3}
 VERIFY_SPLITS = [
     pytest.param(3, 700, 128, 32, 128, 4, 6, "stream", id="streamk-96items-nq16-dh128"),
     pytest.param(3, 700, 128, 32, 128, 6, 12, "stream", id="streamk-96items-nq32-dh128"),
-    pytest.param(3, 700, 128, 32, 128, 8, 20, "stream", id="streamk-96items-nq64-dh128"),
-    pytest.param(3, 700, 128, 32, 64, 8, 20, "stream", id="streamk-96items-nq64-dh64"),
+    pytest.param(3, 700, 128, 32, 128, 8, 20, "stream", id="streamk-96items-nq48-dh128"),
+    pytest.param(3, 700, 128, 32, 128, 8, 26, "stream", id="streamk-96items-nq64-dh128"),
+    pytest.param(3, 700, 128, 32, 64, 8, 20, "stream", id="streamk-96items-nq48-dh64"),
     pytest.param(2, 700, 128, 32, 128, 20, 40, "stream", id="streamk-128items-2chunks-dh128"),
-    pytest.param(5, 1000, 128, 32, 128, 8, 16, "whole", id="whole-160items-nq64-dh128"),
+    pytest.param(5, 1000, 128, 32, 128, 8, 16, "whole", id="whole-160items-nq48-dh128"),
+    pytest.param(5, 1000, 128, 32, 128, 8, 26, "whole", id="whole-160items-nq64-dh128"),
 ]
 
 
