@@ -5,12 +5,21 @@
 namespace fdllm {
 
 size_t proj_workspace_bytes(int M, int D, int H, int dh, int dtype, int num_sms) {
-  if (dtype == FDLLM_BF16) return proj_tc_workspace_bytes(M, D, H, dh, num_sms);
+  if (dtype == FDLLM_BF16) {
+    // a workspace sized for more rows serves fewer: the larger of the two layouts
+    const size_t tc = proj_tc_workspace_bytes(M < kPairMinRows ? M : kPairMinRows - 1, D, H, dh,
+                                              num_sms);
+    const size_t pair = M >= kPairMinRows ? proj_pair_workspace_bytes(M, D, H, dh, num_sms) : 0;
+    return tc > pair ? tc : pair;
+  }
   return proj_simt_workspace_bytes(M, H, dh);
 }
 
 cudaError_t launch_proj(const ProjArgs& a, cudaStream_t stream) {
-  if (a.dtype == FDLLM_BF16) return launch_proj_tc(a, stream);
+  if (a.dtype == FDLLM_BF16) {
+    if (a.B * a.rows_per_seq >= kPairMinRows) return launch_proj_pair(a, stream);
+    return launch_proj_tc(a, stream);
+  }
   return launch_proj_simt(a, stream);
 }
 

@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace fdllm {
@@ -113,6 +114,13 @@ cudaError_t launch_track(const TrackArgs& a, cudaStream_t stream);
 size_t proj_simt_workspace_bytes(int M, int H, int dh);
 size_t proj_tc_workspace_bytes(int M, int D, int H, int dh, int num_sms);
 cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream);
+// bf16 projections of at least kPairMinRows rows run on CTA pairs (below it
+// the single-CTA kernel's split tiles merge faster than the pairs' save)
+constexpr int kPairMinRows = 512;
+size_t proj_pair_workspace_bytes(int M, int D, int H, int dh, int num_sms);
+cudaError_t launch_proj_pair(const ProjArgs& a, cudaStream_t stream);
+// packs x[Q] (rows b, q_idx[m] of x) into xq [M, D] for the fused step
+cudaError_t launch_proj_prep(const ProjArgs& a, __nv_bfloat16* xq, cudaStream_t stream);
 cudaError_t launch_proj_simt(const ProjArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t stream);
 size_t attn_tc_workspace_bytes(int B, int N, int H, int dh, int rows, int S_max, int verify,

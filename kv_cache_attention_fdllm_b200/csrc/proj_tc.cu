@@ -38,6 +38,7 @@
 //               16-byte stores of q, k, v rows
 #include "common.cuh"
 #include "kernels.h"
+#include "proj_epilogue.cuh"
 #include "tc_common.cuh"
 #include "tmap.h"
 
@@ -53,8 +54,6 @@ constexpr int kChunk = 32;          // tokens per epilogue pass
 constexpr int kPitch = kChunk + 1;  // staging pitch (floats)
 constexpr int kMaxBN = 256;
 constexpr uint32_t kASubBytes = kBM * kSub * 2;  // 16 KB
-constexpr double kTwoPi = 6.283185307179586476925286766559;
-constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
 
 
 struct ProjTcParams {
@@ -94,11 +93,6 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* ptr) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
   return v;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 // One CTA per projection row m of the fused step: xq[m] = x[b, q_idx[m]] (zeros
@@ -290,8 +284,6 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     const int quarter = warp & 3;
     const int f_loc = quarter * 32 + lane;
     const int n_half = ((warp - 2) >> 2) * (kChunk / 2);  // this warp's 16 tokens of a chunk
-    const int half = p.dh >> 1;
-    const int dh_log2 = p.dh == 128 ? 7 : 6;  // dh is 64 or 128
     float* my_parts = p.partials + (size_t)c * 2 * BN * kBM;
     int j = 0;
     for (long long u = u_begin; u < u_end; ++j) {
@@ -389,6 +381,20 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           for (int n = etid; n < BN; n += kEpiThreads)
             if (m0 + n < p.M && tok_slot[n] < 0) set_status(p.status, FDLLM_ERR_BAD_INDEX);
         }
+        // The part of contributor cb for this thread's feature row and 16 tokens
+        // from column c (slot 0 when the tile is cb's first: unit_lo(cb) >= tu0).
+        auto load_part = [&](int cb, int c, float* t) {
+          const int sl = (p.total_units * cb >= tu0 * (long long)G) ? 0 : 1;
+          const float* ps = p.partials + ((size_t)cb * 2 + sl) * BN * kBM + (size_t)c * kBM + f_loc;
+#pragma unroll
+          for (int n = 0; n < kChunk / 2; ++n) t[n] = __ldcg(ps + (size_t)n * kBM);
+        };
+        // The first contributor whose part is in global memory has its next
+        // chunk loaded while this chunk is rotated and stored, so the merge
+        // does not wait out an L2 round trip per chunk.
+        const int cb_pf = (c_first == c && own_in_tmem) ? c_first + 1 : c_first;
+        float pf[kChunk / 2];
+        if (!whole && cb_pf <= c_last && n_half < BN) load_part(cb_pf, n_half, pf);
         for (int cc = 0; cc < BN; cc += kChunk) {
           if (whole) {
             // BN is a multiple of 16: a warp's 16 columns are all in the tile or none
@@ -403,6 +409,11 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             // sum the parts of every contributor in CTA (k) order, the thread's
             // feature row over its 16 tokens: this CTA's part from TMEM when it
             // was never stored, the others' from global memory
+            float cur[kChunk / 2];
+#pragma unroll
+            for (int n = 0; n < kChunk / 2; ++n) cur[n] = pf[n];
+            if (cb_pf <= c_last && cc + kChunk + n_half < BN)
+              load_part(cb_pf, cc + kChunk + n_half, pf);
             float v[kChunk / 2];
 #pragma unroll
             for (int n = 0; n < kChunk / 2; ++n) v[n] = 0.f;
@@ -411,13 +422,11 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
               if (cb == c && own_in_tmem) {
                 tc::tmem_ld16(t_acc + cc + n_half, t);
                 tc::tmem_wait_ld();
-              } else {
-                // slot 0 when the tile is cb's first: unit_lo(cb) >= tu0
-                const int sl = (p.total_units * cb >= tu0 * (long long)G) ? 0 : 1;
-                const float* ps = p.partials + ((size_t)cb * 2 + sl) * BN * kBM +
-                                  (size_t)(cc + n_half) * kBM + f_loc;
+              } else if (cb == cb_pf) {
 #pragma unroll
-                for (int n = 0; n < kChunk / 2; ++n) t[n] = __ldcg(ps + (size_t)n * kBM);
+                for (int n = 0; n < kChunk / 2; ++n) t[n] = cur[n];
+              } else {
+                load_part(cb, cc + n_half, t);
               }
 #pragma unroll
               for (int n = 0; n < kChunk / 2; ++n) v[n] += t[n];
@@ -426,61 +435,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             for (int n = 0; n < kChunk / 2; ++n) staging[f_loc * kPitch + n_half + n] = v[n];
           }
           tc::named_bar_sync(1, kEpiThreads);
-          // 32 tokens x 16 groups of 8 features; a warp covers 32 tokens of one group
-          for (int itm = etid; itm < kChunk * (kBM / 8); itm += kEpiThreads) {
-            const int g = itm / kChunk, n = itm % kChunk;
-            const int m = m0 + cc + n;
-            if (cc + n >= BN || m >= p.M) continue;
-            const int f0 = g * 8;
-            const int fg = ft * kBM + f0;
-            if (fg >= p.F) continue;
-            // no integer division: F = 3E and dh is 64 or 128
-            const int blk = fg >= 2 * p.E ? 2 : (fg >= p.E ? 1 : 0);
-            const int rem = fg - blk * p.E;
-            const int h = rem >> dh_log2, j0 = rem & (p.dh - 1);
-            const int slot = tok_slot[cc + n], flag = tok_flag[cc + n];
-            if (blk != 0 && slot < 0) continue;
-            float o[8];
-            if (blk == 2) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) o[i] = staging[(f0 + i) * kPitch + n];
-            } else if (blk == 0 && !(flag & 1)) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) o[i] = 0.f;  // a skipped query attends with q = 0
-            } else {
-              const bool lo = j0 < half;
-              const int pf = lo ? f0 + half : f0 - half;
-              const double* th = theta + (lo ? j0 : j0 - half);
-              const double pos = (double)tok_pos[cc + n];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float x = staging[(f0 + i) * kPitch + n];
-                const float xp = staging[(pf + i) * kPitch + n];
-                // angle mod 2 pi in double, then the fast sine/cosine on [-pi, pi]
-                const double ang = pos * th[i];
-                const double k = rint(ang * kInvTwoPi);
-                float sn, cs;
-                __sincosf((float)fma(-k, kTwoPi, ang), &sn, &cs);
-                o[i] = lo ? (x * cs - xp * sn) : (xp * sn + x * cs);
-              }
-            }
-            uint4 pk;
-            pk.x = pack_bf16x2(o[0], o[1]);
-            pk.y = pack_bf16x2(o[2], o[3]);
-            pk.z = pack_bf16x2(o[4], o[5]);
-            pk.w = pack_bf16x2(o[6], o[7]);
-            __nv_bfloat16* dst;
-            if (blk == 0) {
-              dst = p.q_out + (size_t)m * p.E + h * p.dh + j0;
-            } else {
-              const bool side = (flag & 2) != 0;
-              __nv_bfloat16* base = (blk == 1) ? (side ? p.k_side : p.k_cache)
-                                               : (side ? p.v_side : p.v_cache);
-              const int nslots = side ? p.S_max : p.N;
-              dst = base + (((size_t)tok_b[cc + n] * p.H + h) * nslots + slot) * p.dh + j0;
-            }
-            *reinterpret_cast<uint4*>(dst) = pk;
-          }
+          epi::rope_store_chunk(p, staging, ft * kBM, m0, cc, BN, tok_slot, tok_flag, tok_b, tok_pos,
+                                theta, etid, kEpiThreads);
           tc::named_bar_sync(1, kEpiThreads);
         }
       }
@@ -549,6 +505,14 @@ ProjPlan plan(int M, int D, int H, int dh, int num_sms) {
 
 }  // namespace
 
+cudaError_t launch_proj_prep(const ProjArgs& a, __nv_bfloat16* xq, cudaStream_t stream) {
+  const int M = a.B * a.rows_per_seq;
+  proj_prep_kernel<<<M, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.x), a.idx, a.N, a.D,
+                                          a.rows_per_seq, xq, a.status);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 size_t proj_tc_workspace_bytes(int M, int D, int H, int dh, int num_sms) {
   if (M <= 0) return 256;
   const ProjPlan q = plan(M, D, H, dh, num_sms);
@@ -605,10 +569,7 @@ cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream) {
   cudaError_t e;
   if (!packed) {
     // the fused step gathers x[Q] into a packed operand
-    proj_prep_kernel<<<M, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.x), a.idx, a.N,
-                                            a.D, a.rows_per_seq, xq, a.status);
-    count_launches(1);
-    e = cudaGetLastError();
+    e = launch_proj_prep(a, xq, stream);
     if (e != cudaSuccess) return e;
   }
 

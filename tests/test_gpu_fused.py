@@ -274,3 +274,16 @@ def test_fused_step_rows_reports_repeated_and_out_of_range_indices(F):
         out = torch.empty((2, 3, 128), dtype=torch.bfloat16, device="cuda")
         F.fdllm_fused_step_rows(x_rows, qi, d["w_qkv"], d["k_cache"], d["v_cache"], out, ws)
         assert F.fdllm_get_status(ws) == F.ERR_BAD_INDEX
+
+
+@pytest.mark.parametrize("B,N,D,H,dh,nq", [
+    pytest.param(1, 1200, 128, 2, 128, 512, id="M512-two-token-tiles"),
+    pytest.param(13, 300, 192, 4, 64, 80, id="M1040-five-token-tiles-ragged-k"),
+    pytest.param(6, 500, 256, 5, 128, 100, id="M600-H5-last-pair-past-F"),
+])
+def test_projection_on_cta_pairs(F, B, N, D, H, dh, nq):
+    """512 or more projection rows run on CTA pairs (256 features per MMA, each
+    CTA holding half of the token rows).  The shapes reach token tiles padded
+    past M, several token tiles with a short last k-step, and a last feature
+    pair that runs past F with the q/k block boundary between its two CTAs."""
+    _check_fused(F, W.random_fused(B, N, D, H, dh, nq=nq, seed=91 + nq))

@@ -157,3 +157,11 @@ def test_side_overflow_sets_status(F):
     dev = W.to_device(inp)
     out, ws, st = run_verify_gpu(F, dev, 10000.0)
     assert st == F.ERR_BAD_INDEX
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["mutual", "causal"])
+def test_verify_projection_on_cta_pairs(F, causal):
+    """A verify pass of 520 rows projects on CTA pairs: view-2 rows write side
+    slots, the others cache slots, from both CTAs of a pair."""
+    inp = W.random_verify(13, 400, 128, 4, 64, n_tv=8, n_s=16, seed=73)
+    _check_verify(F, inp, causal=causal)
