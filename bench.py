@@ -410,13 +410,15 @@ def run_ours(args, world, rank, local, cfg=None, name=None, with_e2e=True):
 
     # ---------------- roofline of the dominant kernel
     peak, peak_kind = measured_peaks()
-    alg, _ = algorithmic_bytes(cfg)
+    alg, rows = algorithmic_bytes(cfg)
     stage_mean = {k: sum(v) / len(v) for k, v in stage_ms.items()}
     dom = max(stage_mean, key=stage_mean.get)
     achieved = alg[dom] / (stage_mean[dom] / 1e3) / 1e9
     step_bytes = step_bytes_min(cfg)
     # what the stage call launches, timed together by the events around it
-    kernels = {"proj": "proj_prep_kernel + proj_tc_kernel" if not verify else "proj_tc_kernel",
+    # the library projects 128 rows and more on CTA pairs, fewer on single CTAs
+    proj_k = "proj_pair_kernel" if B * rows >= 128 else "proj_tc_kernel"
+    kernels = {"proj": proj_k if verify else "proj_prep_kernel + " + proj_k,
                "attn": "attn_tc_kernel", "accept": "accept_kernel"}
     if cfg["dtype"] != "bf16":
         kernels = {"proj": "proj_simt kernels", "attn": "attn_simt", "accept": "accept_kernel"}

@@ -114,9 +114,10 @@ cudaError_t launch_track(const TrackArgs& a, cudaStream_t stream);
 size_t proj_simt_workspace_bytes(int M, int H, int dh);
 size_t proj_tc_workspace_bytes(int M, int D, int H, int dh, int num_sms);
 cudaError_t launch_proj_tc(const ProjArgs& a, cudaStream_t stream);
-// bf16 projections of at least kPairMinRows rows run on CTA pairs (below it
-// the single-CTA kernel's split tiles merge faster than the pairs' save)
-constexpr int kPairMinRows = 512;
+// bf16 projections of at least kPairMinRows rows run on CTA pairs.  Below it W
+// is the whole cost and the single-CTA kernel spreads it over every SM, where
+// the pairs' whole tiles leave SMs idle.
+constexpr int kPairMinRows = 128;
 size_t proj_pair_workspace_bytes(int M, int D, int H, int dh, int num_sms);
 cudaError_t launch_proj_pair(const ProjArgs& a, cudaStream_t stream);
 // packs x[Q] (rows b, q_idx[m] of x) into xq [M, D] for the fused step

@@ -8,12 +8,13 @@
 // Y^T [features x tokens] = W_tile * X^T on tcgen05 with cta_group::2: the two
 // CTAs of a cluster share each MMA (M = 256 features, 128 from each CTA's
 // shared memory; N <= 256 tokens, N/2 rows from each), so each CTA loads half
-// of the x[Q] rows a feature tile needs: 32 KB per 64-wide k-step against 48 KB
-// for the single-CTA kernel's 128 x 256 tile, and the L2 -> shared-memory
-// bytes are what bound these shapes.  Two accumulators of up to 256 columns
-// let each tile's epilogue overlap the next tile's MMAs.  (Token tiles of two
-// MMAs, up to 512 tokens in one accumulator, build with FDLLM_PAIR_MAX_BN=512;
-// measured slower: the epilogues between tiles are then exposed.)
+// of the x[Q] rows a feature tile needs, and the L2 -> shared-memory bytes are
+// what bound these shapes.
+//   Up to 512 rows: one token tile (two MMAs of N = BN/2 beyond 256 rows) and,
+//     when there are no more tiles than pairs, one whole tile per pair: W
+//     streams once and no tile is split, so nothing is merged.
+//   More rows: tiles of up to 256 tokens with two accumulators, so that each
+//     tile's epilogue overlaps the next tile's MMAs, spread by stream-K.
 //
 // Both CTAs' TMA loads complete on the rank-0 CTA's stage barrier (the load's
 // cta_group::2 form, no multicast); rank 0 issues the MMAs, and each MMA
@@ -36,9 +37,6 @@
 #include "tc_common.cuh"
 #include "tmap.h"
 
-#ifndef FDLLM_PAIR_MAX_BN
-#define FDLLM_PAIR_MAX_BN 256  // tokens per accumulator
-#endif
 
 namespace fdllm {
 
@@ -50,7 +48,8 @@ constexpr int kThreads = 320;
 constexpr int kEpiThreads = 256;    // two warps per TMEM lane quarter
 constexpr int kChunk = 32;          // tokens per epilogue pass
 constexpr int kPitch = kChunk + 1;  // staging pitch (floats)
-constexpr int kMaxBN = FDLLM_PAIR_MAX_BN;
+constexpr int kMaxBN = 512;         // tokens of one accumulator (two MMAs of N <= 256)
+constexpr int kMaxBNStreamK = 256;  // tokens per tile when tiles outnumber the pairs
 constexpr uint32_t kASubBytes = kBM * kSub * 2;  // 16 KB
 
 struct PairParams {
@@ -484,10 +483,10 @@ int max_pairs(size_t smem_bytes) {
   return cached;
 }
 
-PairPlan plan(int M, int D, int H, int dh, int num_sms, bool resident) {
+PairPlan plan_bn(int M, int D, int H, int dh, int num_sms, bool resident, int max_bn) {
   PairPlan q{};
   const int F = 3 * H * dh;
-  q.n_tt = (M + kMaxBN - 1) / kMaxBN;
+  q.n_tt = (M + max_bn - 1) / max_bn;
   const int per = (M + q.n_tt - 1) / q.n_tt;
   q.BN = ((per + 31) / 32) * 32;
   q.nmma = q.BN > 256 ? 2 : 1;
@@ -523,20 +522,35 @@ PairPlan plan(int M, int D, int H, int dh, int num_sms, bool resident) {
     if (mp > 0 && mp < pairs) pairs = mp;
   }
   if ((long long)pairs > q.total_units) pairs = (int)q.total_units;
+  if (max_bn > kMaxBNStreamK && q.tiles <= pairs) pairs = q.tiles;  // whole tiles
   q.grid = 2 * pairs;
-  // sized by the most columns any row count uses and one pair per two SMs, so
+  // sized by the most columns a split tile has and one pair per two SMs, so
   // that one workspace serves every row count this kernel takes
-  q.partial_bytes = align_up((size_t)(num_sms / 2) * 2 * 2 * kMaxBN * kBM * sizeof(float), 256);
+  q.partial_bytes = align_up((size_t)(num_sms / 2) * 2 * 2 * kMaxBNStreamK * kBM * sizeof(float), 256);
   q.counter_bytes = align_up((size_t)q.tiles * 2 * sizeof(unsigned), 256);
   q.xq_bytes = align_up((size_t)M * D * 2, 256);
   return q;
+}
+
+// Up to 512 rows whose feature tiles fit in one wave of pairs: one token tile
+// (two MMAs beyond 256 rows) and one whole tile per pair, so that W streams
+// once and no tile is split or merged.  Otherwise: tiles of up to 256 tokens
+// with two accumulators, so that each tile's epilogue overlaps the next tile's
+// MMAs, spread over the pairs by stream-K.  The stream-K plan has at least as
+// many tiles as the whole-tile one, so its workspace serves both.
+PairPlan plan(int M, int D, int H, int dh, int num_sms, bool resident) {
+  if (M <= kMaxBN) {
+    PairPlan w = plan_bn(M, D, H, dh, num_sms, resident, kMaxBN);
+    if (2LL * w.tiles == w.grid) return w;
+  }
+  return plan_bn(M, D, H, dh, num_sms, resident, kMaxBNStreamK);
 }
 
 }  // namespace
 
 size_t proj_pair_workspace_bytes(int M, int D, int H, int dh, int num_sms) {
   if (M <= 0) return 256;
-  const PairPlan q = plan(M, D, H, dh, num_sms, false);
+  const PairPlan q = plan_bn(M, D, H, dh, num_sms, false, kMaxBNStreamK);
   return q.partial_bytes + q.counter_bytes + q.xq_bytes;
 }
 

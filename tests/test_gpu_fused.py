@@ -277,13 +277,17 @@ def test_fused_step_rows_reports_repeated_and_out_of_range_indices(F):
 
 
 @pytest.mark.parametrize("B,N,D,H,dh,nq", [
-    pytest.param(1, 1200, 128, 2, 128, 512, id="M512-two-token-tiles"),
+    pytest.param(2, 300, 192, 2, 64, 65, id="M130-whole-tile-one-mma"),
+    pytest.param(3, 400, 128, 3, 128, 100, id="M300-whole-tile-two-mmas-ragged"),
+    pytest.param(2, 500, 256, 5, 128, 100, id="M200-H5-whole-tiles-past-F"),
+    pytest.param(1, 1200, 128, 2, 128, 512, id="M512-whole-tile-two-mmas"),
     pytest.param(13, 300, 192, 4, 64, 80, id="M1040-five-token-tiles-ragged-k"),
     pytest.param(6, 500, 256, 5, 128, 100, id="M600-H5-last-pair-past-F"),
 ])
 def test_projection_on_cta_pairs(F, B, N, D, H, dh, nq):
-    """512 or more projection rows run on CTA pairs (256 features per MMA, each
-    CTA holding half of the token rows).  The shapes reach token tiles padded
+    """128 or more projection rows run on CTA pairs (256 features per MMA, each
+    CTA holding half of the token rows).  Up to 512 rows a pair takes one whole
+    tile of all the rows (two MMAs past 256); the shapes reach a tile padded
     past M, several token tiles with a short last k-step, and a last feature
     pair that runs past F with the q/k block boundary between its two CTAs."""
     _check_fused(F, W.random_fused(B, N, D, H, dh, nq=nq, seed=91 + nq))
