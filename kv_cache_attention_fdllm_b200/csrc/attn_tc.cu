@@ -33,6 +33,15 @@
 //   warp 1      TMEM allocation; lane 0 issues QK (ahead by one tile) and PV
 //   warps 2..   softmax over S^T, P, accumulator rescale, epilogue: NQ/kCols
 //               groups of 4 warps (8 warps at NQ = 32 and 64, 4 at NQ = 16)
+//   last warp   finisher: the item counts of partial segments (stream-K)
+//
+// The O^T accumulator is double-buffered in TMEM by segment (the tiles of one
+// item in a CTA's range), so a segment's end costs the softmax warps only the
+// reduction of l: its output or partial is written two tiles later, once its
+// last PV is long done, while the next segment's PVs accumulate in the other
+// buffer.  A partial's writers signal the finisher, which fences and takes the
+// item count off the softmax warps' path; the items this CTA completes last
+// are merged after its range.
 //
 // Launched as a programmatic dependent: the prologue and an L2 prefetch of
 // the first cache tiles run before the grid-dependency wait; every thread
@@ -55,12 +64,15 @@ constexpr float kThresh = 8.f;  // lazy rescale threshold (log2 units)
 constexpr int kMaxRows = 512;   // verify rows per sequence held in shared memory
 constexpr int kDraftTab = 2048; // cache slots a segment's draft-rank table covers
 constexpr int kL2PrefetchTiles = 4;  // cache tiles per CTA warmed in L2 before the dependency wait
+// the cost of an item boundary inside a stream-K range, in tiles of time
+// (its result is written two tiles later, off the softmax warps' path)
+constexpr double kBoundaryTiles = 1.0;
 // work splits (the values fdllm_attention_split reports)
 constexpr int kSplitStreamK = 1, kSplitWholeItems = 2, kSplitClusters = 3;
 
 struct AttnTcParams {
   int B, N, H, rows, S_max, causal;
-  int n_qc, n_cache_tiles, n_side_tiles, tpi, nk, nv, nqbuf;
+  int n_qc, n_cache_tiles, n_side_tiles, tpi, nk, nv;
   long long total_units;
   float qk_scale;  // log2(e) / sqrt(dh)
   const int32_t* pos;
@@ -77,7 +89,8 @@ struct AttnTcParams {
 };
 
 __device__ __forceinline__ long long unit_lo(long long total, int G, int c) {
-  return total * c / G;
+  const long long a = total * c;
+  return a <= INT_MAX ? (long long)((int)a / G) : a / G;
 }
 // The CTA whose unit range holds unit u: the largest c with unit_lo(c) <= u,
 // i.e. total * c < (u + 1) * G.  A double-precision estimate is corrected with
@@ -91,12 +104,18 @@ __device__ __forceinline__ int owner_of(long long u, long long total, int G) {
   return c;
 }
 
+// a / b for a unit index: 32-bit division when a fits (64-bit integer division
+// is a long software routine)
+__device__ __forceinline__ int unit_div(long long a, int b) {
+  return a <= INT_MAX ? (int)a / b : (int)(a / b);
+}
+
 // (item, tile within the item, query chunk, sequence*head) of a unit, advanced
 // one unit at a time without division.
 struct UnitCursor {
   int item, t, qc, bh;
   __device__ __forceinline__ void init(long long u, int tpi, int n_qc) {
-    item = (int)(u / tpi);
+    item = unit_div(u, tpi);
     t = (int)(u - (long long)item * tpi);
     bh = item / n_qc;
     qc = item - bh * n_qc;
@@ -192,13 +211,19 @@ struct Smem {
 
 // Softmax threads: NQ/kCols groups of 4 warps; a thread owns one key (one dh
 // row) and kCols query columns (16, or 32 at NQ = 64: 256 threads whose
-// registers hold a tile's 32 scores without spilling).
+// registers hold a tile's 32 scores without spilling).  One more warp, the
+// finisher, takes the item counts of the partial segments.
 template <int NQ>
 struct Threads {
   static constexpr int kCols = NQ == 64 ? 32 : 16;
   static constexpr int kSmx = 128 * NQ / kCols;
-  static constexpr int kAll = 64 + kSmx;
+  static constexpr int kFinisher = 2 + kSmx / 32;  // warp index
+  static constexpr int kAll = 64 + kSmx + 32;
 };
+
+// Shared-memory offsets inside the misc block.
+constexpr int kMiscSeg = 4096;    // seg_m[2][64], seg_l[2][64]: (m, l) of a finished segment
+constexpr int kMiscTables = 5120; // verify tables, or the merge weights [8][NQ]
 
 template <int NQ, int DH, bool VERIFY>
 __global__ void __launch_bounds__(Threads<NQ>::kAll, 1)
@@ -214,7 +239,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint8_t* k_ring = smem;
   uint8_t* v_ring = smem + NK * L::kTileBytes;
   uint8_t* q_buf = v_ring + NV * L::kTileBytes;
-  uint8_t* p_buf = q_buf + p.nqbuf * L::kQBytes;  // 1024-aligned (kQBytes is a multiple of 1024)
+  uint8_t* p_buf = q_buf + L::kQBytes;  // 1024-aligned (kQBytes is a multiple of 1024)
   uint8_t* misc = p_buf + 2 * L::kPBufBytes;
   uint64_t* k_full = reinterpret_cast<uint64_t*>(misc);
   uint64_t* k_empty = k_full + 8;
@@ -226,18 +251,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint64_t* s_empty = s_full + 2;    // [2]
   uint64_t* p_full = s_empty + 2;    // [2]
   uint64_t* pv_done = p_full + 2;    // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
+  uint64_t* fin_full = pv_done + 2;  // [2] a partial segment's stores are issued (slot 0, 1)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin_full + 2);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  int* last_flag = abort_flag + 1;
-  int* n_draft_s = last_flag + 1;
+  int* n_draft_s = abort_flag + 1;
   int* n_side_s = n_draft_s + 1;
   int* d_lo_s = n_side_s + 1;  // smallest and largest draft position of the segment
   int* d_hi_s = d_lo_s + 1;
+  int* merge_item = d_hi_s + 1;    // [2] item of partial slot s this CTA merges, or -1
+  int* seg_info = merge_item + 2;  // [2][3] item, first and last tile of a finished segment
   float* m_run = reinterpret_cast<float*>(misc + 512);      // [NQ]
   float* alpha = m_run + 128;                               // [NQ]
   float* wred = alpha + 128;                                // [4][NQ]
   int* col_meta = reinterpret_cast<int*>(wred + 4 * 128);   // [NQ] view | rank << 2
-  int* draft_pos = reinterpret_cast<int*>(misc + 4096);     // [kMaxRows]
+  float* seg_m = reinterpret_cast<float*>(misc + kMiscSeg); // [2][64] (O buffer = segment & 1)
+  float* seg_l = seg_m + 2 * 64;                            // [2][64]
+  int* draft_pos = reinterpret_cast<int*>(misc + kMiscTables);  // [kMaxRows]
   int* draft_rank = draft_pos + kMaxRows;                   // [kMaxRows]
   int* side_rank = draft_rank + kMaxRows;                   // [kMaxRows]
   // draft rank of each cache slot in [d_lo, d_lo + kDraftTab), -1 for no draft
@@ -262,8 +291,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   }
   const int T = (int)(u1 - u0);
 
+  // two S buffers and two O buffers of NQP columns each
   uint32_t ncols = 32;
-  while ((int)ncols < 3 * NQP<NQ>::v) ncols <<= 1;
+  while ((int)ncols < 4 * NQP<NQ>::v) ncols <<= 1;
 
   if (tid == 0) {
     for (int s = 0; s < NK; ++s) {
@@ -283,6 +313,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&p_full[b], kSmx / 32);
       tc::mbar_init(&pv_done[b], 1);
+      tc::mbar_init(&fin_full[b], kSmx / 32);
     }
     *abort_flag = 0;
     tc::fence_mbar_init();
@@ -312,7 +343,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_o = tmem + 2 * NQP<NQ>::v;
+  const uint32_t tmem_o = tmem + 2 * NQP<NQ>::v;  // O buffer b at tmem_o + b * NQP
   // every thread: nothing written by an earlier kernel is read before this
   tc::griddep_wait();
 
@@ -320,35 +351,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // ------------------------------------------------------------ TMA producer
     // K and V have their own rings; each is filled as soon as its stage frees
     // (a K stage right after its QK, a V stage after its PV), polling both so
-    // that neither stream waits behind the other.
+    // that neither stream waits behind the other.  The one Q buffer takes the
+    // next segment's chunk as soon as the last QK of the current one is done.
     if (lane == 0) {
       tc::prefetch_tmap(&tm_q);
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
       const uint64_t pol_kv = tc::policy_evict_first();
       const uint64_t pol_q = tc::policy_evict_last();
-      int ik = 0, iv = 0, seg = -1;
+      const int item_a = unit_div(u0, tpi);
+      const int n_seg = unit_div(u1 - 1, tpi) - item_a + 1;  // segments of this range
+      int ik = 0, iv = 0, qn = 0;
       UnitCursor ck, cv;
       ck.init(u0, tpi, p.n_qc);
       cv = ck;
       IdleClock clk;
-      while (iv < T) {
+      while (iv < T || qn < n_seg) {
         bool progressed = false;
-        if (ik < T) {
-          const int t = ck.t, qc = ck.qc, bh = ck.bh;
-          const bool first = (ik == 0 || t == 0);
-          const int qb = (seg + 1) & 1;
-          const int ks = ik % NK;
-          if (tc::mbar_test(&k_empty[ks], ((uint32_t)(ik / NK) & 1u) ^ 1u) &&
-              (!first || tc::mbar_test(&q_empty[qb], ((uint32_t)((seg + 1) >> 1) & 1u) ^ 1u))) {
-            if (first) {
-              ++seg;
-              tc::mbar_arrive_expect_tx(&q_full[qb], L::kQBytes);
+        if (qn < n_seg && tc::mbar_test(&q_empty[0], ((uint32_t)qn & 1u) ^ 1u)) {
+          const int item = item_a + qn;
+          const int bh = item / p.n_qc, qc = item - bh * p.n_qc;
+          tc::mbar_arrive_expect_tx(&q_full[0], L::kQBytes);
 #pragma unroll
-              for (int x = 0; x < L::kBoxes; ++x)
-                tc::tma_load_4d(q_buf + qb * L::kQBytes + x * NQ * 128, &tm_q, &q_full[qb], x * 64,
-                                bh % p.H, qc * NQ, bh / p.H, pol_q);
-            }
+          for (int x = 0; x < L::kBoxes; ++x)
+            tc::tma_load_4d(q_buf + x * NQ * 128, &tm_q, &q_full[0], x * 64, bh % p.H, qc * NQ,
+                            bh / p.H, pol_q);
+          ++qn;
+          progressed = true;
+        }
+        if (ik < T) {
+          const int ks = ik % NK;
+          if (tc::mbar_test(&k_empty[ks], ((uint32_t)(ik / NK) & 1u) ^ 1u)) {
+            const int t = ck.t, bh = ck.bh;
             const bool side = VERIFY && t >= p.n_cache_tiles;
             const int key0 = (side ? t - p.n_cache_tiles : t) * kKT;
             uint8_t* kd = k_ring + ks * L::kTileBytes;
@@ -390,7 +424,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       constexpr uint32_t idesc_pv = tc::idesc_bf16(kKT, NQ, true, true);
       constexpr uint32_t p_swz = L::kPRow == 128 ? 2u : (L::kPRow == 64 ? 4u : 6u);
       const uint32_t p_addr = tc::smem_u32(p_buf);
-      int iq = 0, ip = 0, seg = -1;
+      int iq = 0, ip = 0, seg = -1, pseg = -1;
       UnitCursor cq, cpv;
       cq.init(u0, tpi, p.n_qc);
       cpv = cq;
@@ -401,16 +435,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const int t = cq.t;
           const bool first = (iq == 0 || t == 0);
           const bool last = (iq == T - 1 || t == tpi - 1);
-          const int qb = first ? ((seg + 1) & 1) : (seg & 1);
           const int qseg = first ? seg + 1 : seg;
           const int ks = iq % NK, sb = iq & 1;
           if (tc::mbar_test(&k_full[ks], (uint32_t)(iq / NK) & 1u) &&
               tc::mbar_test(&s_empty[sb], ((uint32_t)(iq >> 1) & 1u) ^ 1u) &&
-              (!first || tc::mbar_test(&q_full[qb], (uint32_t)(qseg >> 1) & 1u))) {
+              (!first || tc::mbar_test(&q_full[0], (uint32_t)qseg & 1u))) {
             seg = qseg;
             tc::tc_fence_after();
             const uint32_t k_addr = tc::smem_u32(k_ring + ks * L::kTileBytes);
-            const uint32_t q_addr = tc::smem_u32(q_buf + qb * L::kQBytes);
+            const uint32_t q_addr = tc::smem_u32(q_buf);
 #pragma unroll
             for (int kk = 0; kk < DH / 16; ++kk) {
               const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -420,7 +453,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             tc::mma_commit(&s_full[sb]);
             tc::mma_commit(&k_empty[ks]);
-            if (last) tc::mma_commit(&q_empty[qb]);
+            if (last) tc::mma_commit(&q_empty[0]);
             ++iq;
             cq.next(tpi, p.n_qc);
             progressed = true;
@@ -431,14 +464,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           if (tc::mbar_test(&p_full[ip & 1], (uint32_t)(ip >> 1) & 1u) &&
               tc::mbar_test(&v_full[vs], (uint32_t)(ip / NV) & 1u)) {
             const bool first = (ip == 0 || cpv.t == 0);
+            if (first) ++pseg;
             tc::tc_fence_after();
             const uint32_t v_addr = tc::smem_u32(v_ring + vs * L::kTileBytes);
             const uint32_t pb_addr = p_addr + (ip & 1) * L::kPBufBytes;
+            const uint32_t o_addr = tmem_o + (uint32_t)((pseg & 1) * NQP<NQ>::v);
 #pragma unroll
             for (int kk = 0; kk < kKT / 16; ++kk) {
               const uint64_t da = tc::smem_desc(v_addr + kk * 2048, DH == 128 ? 16384 : 0, 1024, 2);
               const uint64_t db = tc::smem_desc(pb_addr + kk * 16 * L::kPRow, 0, 8 * L::kPRow, p_swz);
-              tc::mma_bf16(tmem_o, da, db, idesc_pv, (first && kk == 0) ? 0u : 1u);
+              tc::mma_bf16(o_addr, da, db, idesc_pv, (first && kk == 0) ? 0u : 1u);
             }
             tc::mma_commit(&pv_done[ip & 1]);
             tc::mma_commit(&v_empty[vs]);
@@ -451,7 +486,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (progressed) clk.reset();
       }
     }
-  } else {
+  } else if (warp < Threads<NQ>::kFinisher) {
     // ------------------------------------------------------------ softmax / epilogue
     // NQ/NQH groups of 4 warps: the warps that share a TMEM lane quarter split
     // the query columns, so a thread owns one key (later one dh row) and the
@@ -466,15 +501,81 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const size_t part_floats = (size_t)NQ * DH + 2 * NQ;
     const float scale = p.qk_scale;
     float l[NQH], mrun[NQH];
+#pragma unroll
+    for (int c = 0; c < NQH; ++c) {
+      l[c] = 0.f;
+      mrun[c] = -INFINITY;
+    }
     int seg = -1;
     int n_draft = 0, n_side = 0, d_lo = INT_MAX, d_hi = INT_MIN;
     bool tab = false;      // the segment's draft positions are in kdr_tab
     uint32_t v2cols = 0;   // bit c: this thread's column c0 + c is a mask-view row
-    int pv_waited = -1;  // index of the last PV this thread waited for
-    int seg_t0 = 0;      // tile index at which the current segment started
+    int meta_key = -1;     // (sequence, query chunk) whose verify tables are loaded
+    int pv_waited = -1;    // index of the last PV this thread waited for
+    int seg_t0 = 0;        // tile index at which the current segment started
+    int n_done = 0;        // segments whose last tile is through
+    int n_fin = 0;         // segments whose output or partial is written
+    int end0 = 0, end1 = 0;  // last tile (range index) of the segment in O buffer 0 / 1
     UnitCursor cs;
     cs.init(u0, tpi, p.n_qc);
     const int item0 = cs.item;
+
+    // Writes segment s's result from its O buffer, once its last PV is done:
+    // the output of a whole item, or this CTA's partial (O, m, l) of a split
+    // one, whose arrival on fin_full hands the item count to the finisher.
+    auto finish = [&](int s) {
+      const int sl = s & 1;
+      const int item = seg_info[sl * 3], t0 = seg_info[sl * 3 + 1], tl = seg_info[sl * 3 + 2];
+      const int bh = item / p.n_qc, qc = item - bh * p.n_qc;
+      const int b = bh / p.H, h = bh - b * p.H;
+      const uint32_t t_o = tmem_o + (uint32_t)(sl * NQP<NQ>::v) + lane_off + (uint32_t)c0;
+      const float* sm = seg_m + sl * 64;
+      const float* sls = seg_l + sl * 64;
+      if (t0 == 0 && tl == tpi - 1) {
+#pragma unroll
+        for (int cc = 0; cc < NQH; cc += 16) {
+          float o[16];
+          tc::tmem_ld16(t_o + cc, o);
+          tc::tmem_wait_ld();
+          if (kl < DH) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int cq = c0 + cc + c, r = qc * NQ + cq;
+              if (r < p.rows) {
+                const float lt = sls[cq];
+                p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + kl] = __float2bfloat16_rn(o[c] / lt);
+                if (kl == 0 && p.lse) p.lse[((size_t)b * p.rows + r) * p.H + h] = sm[cq] + log2f(lt);
+              }
+            }
+          }
+        }
+      } else {
+        // slot 0 for the item the range starts in, 1 for the one it ends in
+        // (a split item is only ever one of those two)
+        const int slot = (item == item0) ? 0 : 1;
+        float* part = p.partials + ((size_t)cta * 2 + slot) * part_floats;
+#pragma unroll
+        for (int cc = 0; cc < NQH; cc += 16) {
+          float o[16];
+          tc::tmem_ld16(t_o + cc, o);
+          tc::tmem_wait_ld();
+          if (kl < DH) {
+            // O as [dh row][NQ columns]: a thread's 16 columns are 64 contiguous bytes
+            float4* dst = reinterpret_cast<float4*>(part + (size_t)kl * NQ + c0 + cc);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          }
+        }
+        if (st < NQ) {
+          part[(size_t)NQ * DH + st] = sm[st];
+          part[(size_t)NQ * DH + NQ + st] = sls[st];
+        }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&fin_full[slot]);
+      }
+    };
+
     for (int i = 0; i < T; ++i, cs.next(tpi, p.n_qc)) {
       const int item = cs.item, t = cs.t, qc = cs.qc, bh = cs.bh;
       const bool first = (i == 0 || t == 0);
@@ -483,8 +584,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (first) {
         ++seg;
         seg_t0 = t;
-        // segment metadata: verify tables of sequence b
-        if (VERIFY) {
+        // segment metadata: verify tables of sequence b, query chunk qc (kept
+        // while consecutive segments share them)
+        if (VERIFY && b * p.n_qc + qc != meta_key) {
+          meta_key = b * p.n_qc + qc;
           const int r0 = b * p.rows;
           if (st < NQ) {
             const int r = qc * NQ + st;
@@ -523,14 +626,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               }
             }
           }
-        }
-#pragma unroll
-        for (int c = 0; c < NQH; ++c) {
-          l[c] = 0.f;
-          mrun[c] = -INFINITY;
-        }
-        tc::named_bar_sync(1, kSmx);
-        if (VERIFY) {
+          tc::named_bar_sync(1, kSmx);
           n_draft = *n_draft_s;
           n_side = *n_side_s;
           d_lo = *d_lo_s;
@@ -550,6 +646,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if ((col_meta[c0 + c] & 3) == 2) v2cols |= 1u << c;
         }
       }
+      const uint32_t t_oc = tmem_o + (uint32_t)((seg & 1) * NQP<NQ>::v);  // this segment's O
 
       // ---- raw scores of this tile: row kl of S^T, this thread's columns
       const int sb = i & 1;
@@ -615,8 +712,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
 
       // ---- running max: raised only when a score exceeds it by more than 2^8
-      // (with m = -inf any finite score does; masked scores, -inf, never do)
-      bool need = false;
+      // (with m = -inf any finite score does; masked scores, -inf, never do).
+      // A segment's first tile always sets it, so that no column keeps the
+      // previous segment's max.
+      bool need = first;
 #pragma unroll
       for (int c = 0; c < NQH; ++c) need |= fmaf(s[c], scale, -mrun[c]) > kThresh;
       const bool any = bar_any(2, kSmx, need);
@@ -659,11 +758,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float o[16];
 #pragma unroll
         for (int cc = 0; cc < NQH; cc += 16) {
-          tc::tmem_ld16(tmem_o + lane_off + c0 + cc, o);
+          tc::tmem_ld16(t_oc + lane_off + c0 + cc, o);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 16; ++c) o[c] *= alpha[c0 + cc + c];
-          tc::tmem_st16(tmem_o + lane_off + c0 + cc, o);
+          tc::tmem_st16(t_oc + lane_off + c0 + cc, o);
         }
         tc::tmem_wait_st();
       }
@@ -705,11 +804,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (lane == 0) tc::mbar_arrive(&p_full[i & 1]);
 
       if (last) {
-        // ---- segment done: O^T complete after this tile's PV
-        tc::mbar_wait(&pv_done[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag, p.status);
-        pv_waited = i;
-        tc::tc_fence_after();
-        // total l per column: butterfly within each warp, then across quarters
+        // ---- segment done: l summed per column; (m, l) and the segment's
+        // place are kept for its finish, two tiles on
 #pragma unroll
         for (int c = 0; c < NQH; ++c) {
           float v = l[c];
@@ -720,250 +816,304 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           l[c] = 0.f;
           mrun[c] = -INFINITY;
         }
-        if (st < NQ) alpha[st] = m_run[st];  // keep m while wred is reused below
         tc::named_bar_sync(1, kSmx);
-        float o[NQH];
-        tmem_ld_row<NQH>(tmem_o + lane_off + c0, o);
+        const int sl = seg & 1;
+        if (st < NQ) {
+          seg_m[sl * 64 + st] = m_run[st];
+          seg_l[sl * 64 + st] = wred[st] + wred[NQ + st] + wred[2 * NQ + st] + wred[3 * NQ + st];
+        }
+        if (st == 0) {
+          seg_info[sl * 3] = item;
+          seg_info[sl * 3 + 1] = seg_t0;
+          seg_info[sl * 3 + 2] = t;
+        }
+        if (sl) end1 = i; else end0 = i;
+        ++n_done;
+      }
+
+      // ---- a finished segment writes its result once its last PV is two
+      // tiles back, and at the latest at the end of the segment after it: the
+      // segment two on reuses its O buffer from its first P.  (Kept at the end
+      // of the tile: this code, placed ahead of the scores' wait, slowed each
+      // range's first tile by some microseconds.)
+      while (n_fin < n_done) {
+        const int e = (n_fin & 1) ? end1 : end0;
+        if (!(e <= i - 2 || (last && seg == n_fin + 1))) break;
+        if (pv_waited < e) {
+          tc::mbar_wait(&pv_done[e & 1], (uint32_t)(e >> 1) & 1u, abort_flag, p.status);
+          pv_waited = e;
+        }
+        tc::tc_fence_after();
+        finish(n_fin);
+        ++n_fin;
+      }
+    }
+
+    // ---- the segments not yet finished: the last one or two
+    tc::named_bar_sync(1, kSmx);  // their (m, l) and places are in shared memory
+    if (n_fin < n_done) {
+      if (pv_waited < T - 1) {
+        tc::mbar_wait(&pv_done[(T - 1) & 1], (uint32_t)((T - 1) >> 1) & 1u, abort_flag, p.status);
+        pv_waited = T - 1;
+      }
+      tc::tc_fence_after();
+    }
+    if (clustered) {
+      tc::named_bar_sync(3, kSmx + 32);  // releases the finisher to the cluster barriers
+      // ---- cluster merge of the one segment.  The rings are idle (the last
+      // PV is done), so this CTA's partial goes to the start of the K ring: O^T
+      // as [dh row][NQ + 4] (the pad keeps 16-byte reads of rows at a 144- or
+      // 272-byte stride off each other's banks), then m[NQ], l[NQ].
+      constexpr int kP = NQ + 4;
+      float* cpart = reinterpret_cast<float*>(k_ring);
+#pragma unroll
+      for (int cc = 0; cc < NQH; cc += 16) {
+        float o[16];
+        tc::tmem_ld16(tmem_o + lane_off + c0 + cc, o);
         tc::tmem_wait_ld();
-        const bool whole = (seg_t0 == 0) && (t == tpi - 1);
-        const int h = bh % p.H;
-        if (whole) {
-          if (kl < DH) {
+        if (kl < DH) {
+          float4* dst = reinterpret_cast<float4*>(cpart + kl * kP + c0 + cc);
 #pragma unroll
-            for (int c = 0; c < NQH; ++c) {
-              const int r = qc * NQ + c0 + c;
-              const int cq = c0 + c;
-              if (r < p.rows) {
-                const float lt = wred[cq] + wred[NQ + cq] + wred[2 * NQ + cq] + wred[3 * NQ + cq];
-                p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + kl] = __float2bfloat16_rn(o[c] / lt);
-                if (kl == 0 && p.lse) p.lse[((size_t)b * p.rows + r) * p.H + h] = alpha[cq] + log2f(lt);
-              }
+          for (int v = 0; v < 4; ++v) dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+        }
+      }
+      if (st < NQ) {
+        cpart[DH * kP + st] = seg_m[st];
+        cpart[DH * kP + NQ + st] = seg_l[st];
+      }
+      tc::cluster_sync();
+      const int bh = item0 / p.n_qc, qc = item0 - bh * p.n_qc;
+      const int b = bh / p.H, h = bh - b * p.H;
+      const int cs = p.cs;
+      const uint32_t cbase = tc::smem_u32(cpart);
+      // This CTA merges its slice of dh rows.  A thread takes one row and 4
+      // columns (consecutive threads: consecutive rows, so the output stores
+      // coalesce) and loads (m, l, O) of those columns from up to 4 CTAs at
+      // once, merging online: one round trip per 4 CTAs.
+      const int r0 = (crank * DH) / cs, nr = ((crank + 1) * DH) / cs - r0;
+      for (int idx = st; idx < nr * (NQ / 4); idx += kSmx) {
+        const int row = r0 + idx % nr, c4 = (idx / nr) * 4;
+        float M[4], Lsum[4], acc[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          M[e] = -INFINITY;
+          Lsum[e] = 0.f;
+          acc[e] = 0.f;
+        }
+        for (int g = 0; g < cs; g += 4) {
+          float4 mv[4], lv[4], ov[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (g + j < cs) {
+              const uint32_t a = tc::map_peer(cbase, (uint32_t)(g + j));
+              mv[j] = tc::ld_peer_f32x4(a + (uint32_t)(DH * kP + c4) * 4u);
+              lv[j] = tc::ld_peer_f32x4(a + (uint32_t)(DH * kP + NQ + c4) * 4u);
+              ov[j] = tc::ld_peer_f32x4(a + (uint32_t)(row * kP + c4) * 4u);
+            } else {
+              mv[j] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+              lv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+              ov[j] = lv[j];
             }
           }
-        } else if (clustered) {
-          // ---- cluster merge.  The rings are idle (the last PV is done), so
-          // this CTA's partial goes to the start of the K ring: O^T as
-          // [dh row][NQ + 4] (the pad keeps 16-byte reads of rows at a 144-
-          // or 272-byte stride off each other's banks), then m[NQ], l[NQ].
-          constexpr int kP = NQ + 4;
-          float* cpart = reinterpret_cast<float*>(k_ring);
-          if (kl < DH) {
-            float4* dst = reinterpret_cast<float4*>(cpart + kl * kP + c0);
 #pragma unroll
-            for (int v = 0; v < NQH / 4; ++v)
-              dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
-          }
-          if (st < NQ) {
-            cpart[DH * kP + st] = alpha[st];
-            cpart[DH * kP + NQ + st] = wred[st] + wred[NQ + st] + wred[2 * NQ + st] + wred[3 * NQ + st];
-          }
-          tc::cluster_sync();
-          const int cs = p.cs;
-          const uint32_t cbase = tc::smem_u32(cpart);
-          // This CTA merges its slice of dh rows.  A thread takes one row and 4
-          // columns (consecutive threads: consecutive rows, so the output
-          // stores coalesce) and loads (m, l, O) of those columns from up to 4
-          // CTAs at once, merging online: one round trip per 4 CTAs.
-          const int r0 = (crank * DH) / cs, nr = ((crank + 1) * DH) / cs - r0;
-          for (int idx = st; idx < nr * (NQ / 4); idx += kSmx) {
-            const int row = r0 + idx % nr, c4 = (idx / nr) * 4;
-            float M[4], Lsum[4], acc[4];
+          for (int e = 0; e < 4; ++e) {
+            float mj[4], lj[4], oj[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              M[e] = -INFINITY;
-              Lsum[e] = 0.f;
-              acc[e] = 0.f;
+            for (int j = 0; j < 4; ++j) {
+              mj[j] = e == 0 ? mv[j].x : e == 1 ? mv[j].y : e == 2 ? mv[j].z : mv[j].w;
+              lj[j] = e == 0 ? lv[j].x : e == 1 ? lv[j].y : e == 2 ? lv[j].z : lv[j].w;
+              oj[j] = e == 0 ? ov[j].x : e == 1 ? ov[j].y : e == 2 ? ov[j].z : ov[j].w;
             }
-            for (int g = 0; g < cs; g += 4) {
-              float4 mv[4], lv[4], ov[4];
+            const float mn = fmaxf(fmaxf(M[e], fmaxf(mj[0], mj[1])), fmaxf(mj[2], mj[3]));
+            if (mn > -INFINITY) {
+              const float sc = (M[e] == -INFINITY) ? 0.f : exp2f(M[e] - mn);
+              Lsum[e] *= sc;
+              acc[e] *= sc;
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                if (g + j < cs) {
-                  const uint32_t a = tc::map_peer(cbase, (uint32_t)(g + j));
-                  mv[j] = tc::ld_peer_f32x4(a + (uint32_t)(DH * kP + c4) * 4u);
-                  lv[j] = tc::ld_peer_f32x4(a + (uint32_t)(DH * kP + NQ + c4) * 4u);
-                  ov[j] = tc::ld_peer_f32x4(a + (uint32_t)(row * kP + c4) * 4u);
-                } else {
-                  mv[j] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-                  lv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-                  ov[j] = lv[j];
-                }
+                const float w = (mj[j] == -INFINITY) ? 0.f : exp2f(mj[j] - mn);
+                Lsum[e] = fmaf(w, lj[j], Lsum[e]);
+                acc[e] = fmaf(w, oj[j], acc[e]);
               }
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                float mj[4], lj[4], oj[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  mj[j] = e == 0 ? mv[j].x : e == 1 ? mv[j].y : e == 2 ? mv[j].z : mv[j].w;
-                  lj[j] = e == 0 ? lv[j].x : e == 1 ? lv[j].y : e == 2 ? lv[j].z : lv[j].w;
-                  oj[j] = e == 0 ? ov[j].x : e == 1 ? ov[j].y : e == 2 ? ov[j].z : ov[j].w;
-                }
-                const float mn = fmaxf(fmaxf(M[e], fmaxf(mj[0], mj[1])), fmaxf(mj[2], mj[3]));
-                if (mn > -INFINITY) {
-                  const float sc = (M[e] == -INFINITY) ? 0.f : exp2f(M[e] - mn);
-                  Lsum[e] *= sc;
-                  acc[e] *= sc;
-#pragma unroll
-                  for (int j = 0; j < 4; ++j) {
-                    const float w = (mj[j] == -INFINITY) ? 0.f : exp2f(mj[j] - mn);
-                    Lsum[e] = fmaf(w, lj[j], Lsum[e]);
-                    acc[e] = fmaf(w, oj[j], acc[e]);
-                  }
-                  M[e] = mn;
-                }
-              }
-            }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int r = qc * NQ + c4 + e;
-              if (r < p.rows) {
-                p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + row] =
-                    __float2bfloat16_rn(Lsum[e] > 0.f ? acc[e] / Lsum[e] : 0.f);
-                if (row == 0 && p.lse) p.lse[((size_t)b * p.rows + r) * p.H + h] = M[e] + log2f(Lsum[e]);
-              }
-            }
-          }
-          // no CTA leaves while another may still read its shared memory
-          tc::cluster_sync();
-        } else {
-          // partial item: (O, m, l) to this CTA's slot; the last contributor merges.
-          // Slot: O as [dh row][NQ columns] (a thread's 16 columns are 64
-          // contiguous bytes), then m[NQ], then l[NQ].
-          const int slot = (item == item0) ? 0 : 1;
-          float* part = p.partials + ((size_t)cta * 2 + slot) * part_floats;
-          if (kl < DH) {
-            float4* dst = reinterpret_cast<float4*>(part + (size_t)kl * NQ + c0);
-#pragma unroll
-            for (int v = 0; v < NQH / 4; ++v)
-              dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
-          }
-          if (st < NQ) {
-            part[(size_t)NQ * DH + st] = alpha[st];
-            part[(size_t)NQ * DH + NQ + st] = wred[st] + wred[NQ + st] + wred[2 * NQ + st] + wred[3 * NQ + st];
-          }
-          __threadfence();
-          tc::named_bar_sync(1, kSmx);
-          const long long iu0 = (long long)item * tpi;
-          const int c_first = owner_of(iu0, p.total_units, G);
-          const int c_last = owner_of(iu0 + tpi - 1, p.total_units, G);
-          if (st == 0) {
-            const unsigned prev = atomicAdd(&p.item_cnt[item], 1u);
-            *last_flag = (prev == (unsigned)(c_last - c_first));
-            if (*last_flag) p.item_cnt[item] = 0u;
-          }
-          tc::named_bar_sync(1, kSmx);
-          if (*last_flag) {
-            __threadfence();
-            // Merge the contributors in CTA order.  The loads of a batch are
-            // all issued before any is used, so the merge costs a few L2 round
-            // trips, not a few per contributor.
-            //   (1) per column: M = max m_j, L = sum 2^(m_j - M) l_j (8 at a time)
-            //   (2) O = sum (2^(m_j - M) / L) O_j, weights staged in shared memory
-            const int n_c = c_last - c_first + 1;
-            // slot 0 when the item is the contributor's first, i.e. its range
-            // starts inside the item: unit_lo(cb) >= iu0 <=> total * cb >= iu0 * G
-            const long long lim0 = iu0 * (long long)G;
-            auto part_of = [&](int cb) -> const float* {
-              const int sl = (p.total_units * cb >= lim0) ? 0 : 1;
-              return p.partials + ((size_t)cb * 2 + sl) * part_floats;
-            };
-            float* wts = reinterpret_cast<float*>(draft_pos);  // [8][NQ], free here
-            float M = -INFINITY, Lsum = 0.f;
-            float mv[8];
-            if (st < NQ) {
-              for (int g0 = 0; g0 < n_c; g0 += 8) {
-                float lv[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                  mv[j] = -INFINITY;
-                  lv[j] = 0.f;
-                  if (g0 + j < n_c) {
-                    const float* pc = part_of(c_first + g0 + j);
-                    mv[j] = __ldcg(pc + (size_t)NQ * DH + st);
-                    lv[j] = __ldcg(pc + (size_t)NQ * DH + NQ + st);
-                  }
-                }
-                float mc = M;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) mc = fmaxf(mc, mv[j]);
-                if (mc > -INFINITY) {
-                  Lsum *= (M == -INFINITY) ? 0.f : exp2f(M - mc);
-#pragma unroll
-                  for (int j = 0; j < 8; ++j) Lsum += (mv[j] == -INFINITY) ? 0.f : exp2f(mv[j] - mc) * lv[j];
-                  M = mc;
-                }
-              }
-            }
-            if (st < NQ && p.lse && qc * NQ + st < p.rows)
-              p.lse[((size_t)b * p.rows + qc * NQ + st) * p.H + h] = M + log2f(Lsum);
-            constexpr int kJ = NQH == 32 ? 2 : 4;  // contributors per batch of O loads
-            float acc[NQH];
-#pragma unroll
-            for (int c = 0; c < NQH; ++c) acc[c] = 0.f;
-            for (int g0 = 0; g0 < n_c; g0 += 8) {
-              if (st < NQ) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                  float m = mv[j];
-                  if (n_c > 8) m = (g0 + j < n_c) ? __ldcg(part_of(c_first + g0 + j) + (size_t)NQ * DH + st) : -INFINITY;
-                  wts[j * NQ + st] = (m == -INFINITY || !(Lsum > 0.f)) ? 0.f : exp2f(m - M) / Lsum;
-                }
-              }
-              tc::named_bar_sync(1, kSmx);
-              if (kl < DH) {
-                const int nj = min(8, n_c - g0);
-                for (int j0 = 0; j0 < nj; j0 += kJ) {
-                  float4 ov[kJ][NQH / 4];
-#pragma unroll
-                  for (int j = 0; j < kJ; ++j) {
-                    if (j0 + j < nj) {
-                      const float4* src = reinterpret_cast<const float4*>(part_of(c_first + g0 + j0 + j) + (size_t)kl * NQ + c0);
-#pragma unroll
-                      for (int v = 0; v < NQH / 4; ++v) ov[j][v] = __ldcg(src + v);
-                    } else {
-#pragma unroll
-                      for (int v = 0; v < NQH / 4; ++v) ov[j][v] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-                  }
-#pragma unroll
-                  for (int j = 0; j < kJ; ++j) {
-                    const float* wj = wts + (j0 + j) * NQ + c0;
-#pragma unroll
-                    for (int v = 0; v < NQH / 4; ++v) {
-                      // weights past nj are stale but multiply zeros
-                      const float w0 = (j0 + j < nj) ? wj[4 * v] : 0.f;
-                      const float w1 = (j0 + j < nj) ? wj[4 * v + 1] : 0.f;
-                      const float w2 = (j0 + j < nj) ? wj[4 * v + 2] : 0.f;
-                      const float w3 = (j0 + j < nj) ? wj[4 * v + 3] : 0.f;
-                      acc[4 * v] = fmaf(w0, ov[j][v].x, acc[4 * v]);
-                      acc[4 * v + 1] = fmaf(w1, ov[j][v].y, acc[4 * v + 1]);
-                      acc[4 * v + 2] = fmaf(w2, ov[j][v].z, acc[4 * v + 2]);
-                      acc[4 * v + 3] = fmaf(w3, ov[j][v].w, acc[4 * v + 3]);
-                    }
-                  }
-                }
-              }
-              tc::named_bar_sync(1, kSmx);
-            }
-            if (kl < DH) {
-#pragma unroll
-              for (int c = 0; c < NQH; ++c) {
-                const int r = qc * NQ + c0 + c;
-                if (r < p.rows)
-                  p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + kl] = __float2bfloat16_rn(acc[c]);
-              }
+              M[e] = mn;
             }
           }
         }
-        tc::tc_fence_before();
-        tc::named_bar_sync(1, kSmx);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = qc * NQ + c4 + e;
+          if (r < p.rows) {
+            p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + row] =
+                __float2bfloat16_rn(Lsum[e] > 0.f ? acc[e] / Lsum[e] : 0.f);
+            if (row == 0 && p.lse) p.lse[((size_t)b * p.rows + r) * p.H + h] = M[e] + log2f(Lsum[e]);
+          }
+        }
       }
+      // no CTA leaves while another may still read its shared memory
+      tc::cluster_sync();
+    } else {
+      while (n_fin < n_done) {
+        finish(n_fin);
+        ++n_fin;
+      }
+      // the finisher has taken the counts of this CTA's partial segments
+      tc::named_bar_sync(3, kSmx + 32);
+      for (int slot = 0; slot < 2; ++slot) {
+        const int item = merge_item[slot];
+        if (item < 0) continue;
+        // ---- merge item `item`, whose contributors have all stored their
+        // partials, in CTA order.  The loads of a batch are all issued before
+        // any is used, so the merge costs a few L2 round trips, not a few per
+        // contributor.
+        //   (1) per column: M = max m_j, L = sum 2^(m_j - M) l_j (8 at a time)
+        //   (2) O = sum (2^(m_j - M) / L) O_j, weights staged in shared memory
+        __threadfence();
+        const int bh = item / p.n_qc, qc = item - bh * p.n_qc;
+        const int b = bh / p.H, h = bh - b * p.H;
+        const long long iu0 = (long long)item * tpi;
+        const int c_first = owner_of(iu0, p.total_units, G);
+        const int c_last = owner_of(iu0 + tpi - 1, p.total_units, G);
+        const int n_c = c_last - c_first + 1;
+        // slot 0 when the item is the contributor's first, i.e. its range
+        // starts inside the item: unit_lo(cb) >= iu0 <=> total * cb >= iu0 * G
+        const long long lim0 = iu0 * (long long)G;
+        auto part_of = [&](int cb) -> const float* {
+          const int sl = (p.total_units * cb >= lim0) ? 0 : 1;
+          return p.partials + ((size_t)cb * 2 + sl) * part_floats;
+        };
+        float* wts = reinterpret_cast<float*>(draft_pos);  // [8][NQ], free after the range
+        float M = -INFINITY, Lsum = 0.f;
+        float mv[8];
+        if (st < NQ) {
+          for (int g0 = 0; g0 < n_c; g0 += 8) {
+            float lv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              mv[j] = -INFINITY;
+              lv[j] = 0.f;
+              if (g0 + j < n_c) {
+                const float* pc = part_of(c_first + g0 + j);
+                mv[j] = __ldcg(pc + (size_t)NQ * DH + st);
+                lv[j] = __ldcg(pc + (size_t)NQ * DH + NQ + st);
+              }
+            }
+            float mc = M;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mc = fmaxf(mc, mv[j]);
+            if (mc > -INFINITY) {
+              Lsum *= (M == -INFINITY) ? 0.f : exp2f(M - mc);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) Lsum += (mv[j] == -INFINITY) ? 0.f : exp2f(mv[j] - mc) * lv[j];
+              M = mc;
+            }
+          }
+        }
+        if (st < NQ && p.lse && qc * NQ + st < p.rows)
+          p.lse[((size_t)b * p.rows + qc * NQ + st) * p.H + h] = M + log2f(Lsum);
+        constexpr int kJ = NQH == 32 ? 2 : 4;  // contributors per batch of O loads
+        float acc[NQH];
+#pragma unroll
+        for (int c = 0; c < NQH; ++c) acc[c] = 0.f;
+        for (int g0 = 0; g0 < n_c; g0 += 8) {
+          if (st < NQ) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float m = mv[j];
+              if (n_c > 8) m = (g0 + j < n_c) ? __ldcg(part_of(c_first + g0 + j) + (size_t)NQ * DH + st) : -INFINITY;
+              wts[j * NQ + st] = (m == -INFINITY || !(Lsum > 0.f)) ? 0.f : exp2f(m - M) / Lsum;
+            }
+          }
+          tc::named_bar_sync(1, kSmx);
+          if (kl < DH) {
+            const int nj = min(8, n_c - g0);
+            for (int j0 = 0; j0 < nj; j0 += kJ) {
+              float4 ov[kJ][NQH / 4];
+#pragma unroll
+              for (int j = 0; j < kJ; ++j) {
+                if (j0 + j < nj) {
+                  const float4* src = reinterpret_cast<const float4*>(part_of(c_first + g0 + j0 + j) + (size_t)kl * NQ + c0);
+#pragma unroll
+                  for (int v = 0; v < NQH / 4; ++v) ov[j][v] = __ldcg(src + v);
+                } else {
+#pragma unroll
+                  for (int v = 0; v < NQH / 4; ++v) ov[j][v] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+              }
+#pragma unroll
+              for (int j = 0; j < kJ; ++j) {
+                const float* wj = wts + (j0 + j) * NQ + c0;
+#pragma unroll
+                for (int v = 0; v < NQH / 4; ++v) {
+                  // weights past nj are stale but multiply zeros
+                  const float w0 = (j0 + j < nj) ? wj[4 * v] : 0.f;
+                  const float w1 = (j0 + j < nj) ? wj[4 * v + 1] : 0.f;
+                  const float w2 = (j0 + j < nj) ? wj[4 * v + 2] : 0.f;
+                  const float w3 = (j0 + j < nj) ? wj[4 * v + 3] : 0.f;
+                  acc[4 * v] = fmaf(w0, ov[j][v].x, acc[4 * v]);
+                  acc[4 * v + 1] = fmaf(w1, ov[j][v].y, acc[4 * v + 1]);
+                  acc[4 * v + 2] = fmaf(w2, ov[j][v].z, acc[4 * v + 2]);
+                  acc[4 * v + 3] = fmaf(w3, ov[j][v].w, acc[4 * v + 3]);
+                }
+              }
+            }
+          }
+          tc::named_bar_sync(1, kSmx);
+        }
+        if (kl < DH) {
+#pragma unroll
+          for (int c = 0; c < NQH; ++c) {
+            const int r = qc * NQ + c0 + c;
+            if (r < p.rows)
+              p.out[(((size_t)b * p.rows + r) * p.H + h) * DH + kl] = __float2bfloat16_rn(acc[c]);
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ finisher
+    // For each partial segment of this CTA's range, in order: wait until the
+    // softmax warps have issued its stores, make them visible device-wide,
+    // then count this contributor in.  The last of an item's contributors
+    // merges it; the softmax warps do that after the range.
+    if (!clustered) {
+      if (lane == 0) {
+        merge_item[0] = -1;
+        merge_item[1] = -1;
+        const int item_a = unit_div(u0, tpi), item_z = unit_div(u1 - 1, tpi);
+        for (int slot = 0; slot < 2; ++slot) {
+          const int item = slot == 0 ? item_a : item_z;
+          if (slot == 1 && item_z == item_a) break;
+          const long long iu0 = (long long)item * tpi;
+          if (u0 <= iu0 && u1 >= iu0 + tpi) continue;  // whole: the softmax warps write it
+          // polled with a pause between tests, so that this warp takes no issue
+          // slots from the softmax warps of its SM sub-partition meanwhile
+          bool ready = false;
+          IdleClock clk;
+          while (!(ready = tc::mbar_test(&fin_full[slot], 0u))) {
+            __nanosleep(256);
+            if (!clk.idle(abort_flag, p.status)) break;
+          }
+          if (!ready) break;
+          __threadfence();
+          const int c_first = owner_of(iu0, p.total_units, G);
+          const int c_last = owner_of(iu0 + tpi - 1, p.total_units, G);
+          const unsigned prev = atomicAdd(&p.item_cnt[item], 1u);
+          if (prev == (unsigned)(c_last - c_first)) {
+            p.item_cnt[item] = 0u;  // reset for the next call
+            merge_item[slot] = item;
+          }
+        }
+      }
+      __syncwarp();
+      tc::named_bar_sync(3, kSmx + 32);
     }
   }
 
-  // the softmax warps meet the two cluster barriers of the merge; the producer
-  // and MMA warps, done with their loops, meet them here
-  if (clustered && warp < 2) {
+  // the softmax warps meet the two cluster barriers of the merge; the other
+  // warps, done with their loops, meet them here (the finisher once the merge
+  // begins: it waits on a CTA barrier, not a cluster one, meanwhile)
+  if (clustered && (warp < 2 || warp == Threads<NQ>::kFinisher)) {
+    if (warp == Threads<NQ>::kFinisher) tc::named_bar_sync(3, kSmx + 32);
     tc::cluster_sync();
     tc::cluster_sync();
   }
@@ -977,11 +1127,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 }
 
 struct AttnPlan {
-  int NQ, n_qc, nct, nst, tpi, nk, nv, grid;  // stream-K: rings, grid
-  int cs, nk_cl, nv_cl;                        // cluster size wanted (0: stream-K), its rings
+  int NQ, n_qc, nct, nst, tpi, nk, nv, grid;  // rings; stream-K grid
+  int cs;                                      // cluster size wanted (0: none)
   bool whole_items;                            // many items: one CTA per item, no merges
   long long items, total_units;
-  size_t smem_bytes, smem_cl, partial_bytes, counter_bytes;
+  size_t smem_bytes, partial_bytes, counter_bytes;
 };
 
 constexpr size_t kSmemBudget = 227 * 1024;
@@ -1009,34 +1159,28 @@ AttnPlan plan(int B, int N, int H, int dh, int rows, int S_max, int verify, int 
   const size_t qbytes = boxes * q.NQ * 128;
   const size_t nqp = q.NQ == 48 ? 64 : q.NQ;  // P's padded columns
   const size_t pbytes = 2 * (((size_t)kKT * nqp * 2 + 1023) / 1024 * 1024);
-  // misc: barriers and softmax scratch, then the verify tables (or, without
-  // them, the [8][NQ] merge weights of the stream-K path)
-  const size_t misc = 4096 + (verify ? 3 * kMaxRows * 4 + kDraftTab * 2 : 8 * 64 * 4);
+  // misc: barriers, softmax scratch and the finished segments' (m, l), then the
+  // verify tables (or, without them, the [8][NQ] merge weights)
+  const size_t misc = kMiscTables + (verify ? 3 * kMaxRows * 4 + kDraftTab * 2 : 8 * 64 * 4);
   // K and V tiles share what shared memory is left.  A V tile is held from its
   // load until its PV is done, longer than a K tile, so V gets the odd one.
-  // Cluster mode runs one item per CTA and needs one Q buffer, not two.
-  auto rings = [&](int nqbuf, int& nk, int& nv) -> size_t {
-    const size_t fixed = 1024 + nqbuf * qbytes + pbytes + misc;
-    int tiles = (int)((kSmemBudget - fixed) / tile);
-    if (tiles > 16) tiles = 16;
-    nv = (tiles + 1) / 2;
-    nk = tiles - nv;
-    if (nv > 8) nv = 8;
-    return fixed + (size_t)(nk + nv) * tile;
-  };
-  q.smem_bytes = rings(2, q.nk, q.nv);
-  q.smem_cl = rings(1, q.nk_cl, q.nv_cl);
-  // Many items in at most two waves: one CTA per whole item avoids the item
-  // boundaries inside a CTA's range - each costs the softmax warps an epilogue
-  // and a new item's setup while the next tile waits, about 6 tiles of time -
-  // and every merge.  Taken when its wave-quantised makespan is no longer than
-  // stream-K's plus two such boundaries.  With more waves every CTA's cold
+  const size_t fixed = 1024 + qbytes + pbytes + misc;
+  int tiles = (int)((kSmemBudget - fixed) / tile);
+  if (tiles > 16) tiles = 16;
+  q.nv = (tiles + 1) / 2;
+  q.nk = tiles - q.nv;
+  if (q.nv > 8) q.nv = 8;
+  q.smem_bytes = fixed + (size_t)(q.nk + q.nv) * tile;
+  // Many items in at most two waves: one CTA per whole item has no item
+  // boundary inside a CTA's range and no merge.  Taken when its
+  // wave-quantised makespan is no longer than stream-K's plus two boundaries,
+  // each about kBoundaryTiles of tile time.  With more waves every CTA's cold
   // start (about 5 us) adds up, and persistent stream-K, which pipelines its
   // loads across item boundaries, wins (measured: 2048 items, 649 -> 705 us).
   q.whole_items = false;
   if (q.cs == 0 && q.items > num_sms) {
     const long long waves = (q.items + num_sms - 1) / num_sms;
-    const double sk_tiles = (double)q.total_units / num_sms + 2 * 6.0;
+    const double sk_tiles = (double)q.total_units / num_sms + 2 * kBoundaryTiles;
     q.whole_items = waves <= 2 && (double)(waves * q.tpi) <= sk_tiles;
   }
   q.partial_bytes = align_up((size_t)q.grid * 2 * ((size_t)q.NQ * dh + 2 * q.NQ) * sizeof(float), 256);
@@ -1076,12 +1220,11 @@ int max_clusters(int cs, size_t smem_bytes) {
 template <int NQ, int DH, bool VERIFY>
 cudaError_t resolve_split(const AttnPlan& q, int* mode, int* cs_out) {
   auto kern = attn_tc_kernel<NQ, DH, VERIFY>;
-  const size_t smem_max = q.smem_bytes > q.smem_cl ? q.smem_bytes : q.smem_cl;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem_max);
+                                       (int)q.smem_bytes);
   if (e != cudaSuccess) return e;
   int cs = q.cs;
-  while (cs >= 2 && max_clusters<NQ, DH, VERIFY>(cs, q.smem_cl) < q.items) --cs;
+  while (cs >= 2 && max_clusters<NQ, DH, VERIFY>(cs, q.smem_bytes) < q.items) --cs;
   if (cs >= 2) {
     *mode = kSplitClusters;
     *cs_out = cs;
@@ -1114,27 +1257,18 @@ cudaError_t launch_t(const AttnArgs& a, const AttnPlan& q, AttnTcParams prm, con
     attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
     cfg.gridDim = dim3((unsigned)(q.items * cs));
-    cfg.dynamicSmemBytes = q.smem_cl;
     prm.cs = cs;
-    prm.nk = q.nk_cl;
-    prm.nv = q.nv_cl;
-    prm.nqbuf = 1;
   } else if (mode == kSplitWholeItems) {
     // grid = items: the unit split gives every CTA exactly one whole item
     cfg.gridDim = dim3((unsigned)q.items);
-    cfg.dynamicSmemBytes = q.smem_cl;
     prm.cs = 0;
-    prm.nk = q.nk_cl;
-    prm.nv = q.nv_cl;
-    prm.nqbuf = 1;
   } else {
     cfg.gridDim = dim3(q.grid);
-    cfg.dynamicSmemBytes = q.smem_bytes;
     prm.cs = 0;
-    prm.nk = q.nk;
-    prm.nv = q.nv;
-    prm.nqbuf = 2;
   }
+  cfg.dynamicSmemBytes = q.smem_bytes;
+  prm.nk = q.nk;
+  prm.nv = q.nv;
   e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], prm);
   count_launches(1);
   return e;

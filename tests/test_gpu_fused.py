@@ -83,10 +83,14 @@ def test_ragged_shapes(F, dtype, dh, shape):
 # 2 SMs when its two waves are no slower than stream-K; stream-K takes the rest
 # above SMs / 2.
 SPLIT_SHAPES = [
-    pytest.param(5, 1000, 128, 32, 64, 20, "whole", id="whole-160items-nq32-dh64"),
-    pytest.param(12, 700, 128, 16, 128, 12, "whole", id="whole-192items-nq16-dh128"),
-    pytest.param(8, 1024, 128, 32, 128, 32, "whole", id="whole-256items-nq32-dh128"),
-    pytest.param(5, 1000, 128, 32, 128, 40, "whole", id="whole-160items-nq48-dh128"),
+    pytest.param(9, 1000, 128, 32, 64, 20, "whole", id="whole-288items-nq32-dh64"),
+    pytest.param(9, 700, 128, 32, 128, 12, "whole", id="whole-288items-nq16-dh128"),
+    pytest.param(9, 1024, 128, 32, 128, 32, "whole", id="whole-288items-nq32-dh128"),
+    pytest.param(9, 1000, 128, 32, 128, 40, "whole", id="whole-288items-nq48-dh128"),
+    pytest.param(5, 1000, 128, 32, 64, 20, "stream", id="streamk-160items-nq32-dh64"),
+    pytest.param(12, 700, 128, 16, 128, 12, "stream", id="streamk-192items-nq16-dh128"),
+    pytest.param(8, 1024, 128, 32, 128, 32, "stream", id="streamk-256items-nq32-dh128"),
+    pytest.param(5, 1000, 128, 32, 128, 40, "stream", id="streamk-160items-nq48-dh128"),
     pytest.param(3, 900, 128, 32, 128, 60, "stream", id="streamk-96items-nq64-dh128"),
     pytest.param(3, 900, 128, 32, 64, 44, "stream", id="streamk-96items-nq48-dh64"),
     pytest.param(12, 600, 128, 32, 64, 30, "stream", id="streamk-384items-nq32-dh64"),

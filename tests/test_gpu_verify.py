@@ -74,8 +74,10 @@ VERIFY_SPLITS = [
     pytest.param(3, 700, 128, 32, 128, 8, 26, "stream", id="streamk-96items-nq64-dh128"),
     pytest.param(3, 700, 128, 32, 64, 8, 20, "stream", id="streamk-96items-nq48-dh64"),
     pytest.param(2, 700, 128, 32, 128, 20, 40, "stream", id="streamk-128items-2chunks-dh128"),
-    pytest.param(5, 1000, 128, 32, 128, 8, 16, "whole", id="whole-160items-nq48-dh128"),
-    pytest.param(5, 1000, 128, 32, 128, 8, 26, "whole", id="whole-160items-nq64-dh128"),
+    pytest.param(5, 1000, 128, 32, 128, 8, 16, "stream", id="streamk-160items-nq48-dh128"),
+    pytest.param(5, 1000, 128, 32, 128, 8, 26, "stream", id="streamk-160items-nq64-dh128"),
+    pytest.param(9, 1000, 128, 32, 128, 8, 16, "whole", id="whole-288items-nq48-dh128"),
+    pytest.param(9, 1000, 128, 32, 128, 8, 26, "whole", id="whole-288items-nq64-dh128"),
 ]
 
 
