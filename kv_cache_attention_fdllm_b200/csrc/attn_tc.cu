@@ -64,9 +64,13 @@ constexpr float kThresh = 8.f;  // lazy rescale threshold (log2 units)
 constexpr int kMaxRows = 512;   // verify rows per sequence held in shared memory
 constexpr int kDraftTab = 2048; // cache slots a segment's draft-rank table covers
 constexpr int kL2PrefetchTiles = 4;  // cache tiles per CTA warmed in L2 before the dependency wait
-// the cost of an item boundary inside a stream-K range, in tiles of time
-// (its result is written two tiles later, off the softmax warps' path)
+// Costs in tiles of time, for choosing between one CTA per whole item and
+// stream-K: an item boundary inside a stream-K range (its result is written
+// later, off the softmax warps' path), a CTA's cold start, and the merge of the
+// items a stream-K CTA completes last
 constexpr double kBoundaryTiles = 1.0;
+constexpr double kStartTiles = 3.0;
+constexpr double kMergeTiles = 3.0;
 // work splits (the values fdllm_attention_split reports)
 constexpr int kSplitStreamK = 1, kSplitWholeItems = 2, kSplitClusters = 3;
 
@@ -1171,17 +1175,18 @@ AttnPlan plan(int B, int N, int H, int dh, int rows, int S_max, int verify, int 
   q.nk = tiles - q.nv;
   if (q.nv > 8) q.nv = 8;
   q.smem_bytes = fixed + (size_t)(q.nk + q.nv) * tile;
-  // Many items in at most two waves: one CTA per whole item has no item
-  // boundary inside a CTA's range and no merge.  Taken when its
-  // wave-quantised makespan is no longer than stream-K's plus two boundaries,
-  // each about kBoundaryTiles of tile time.  With more waves every CTA's cold
-  // start (about 5 us) adds up, and persistent stream-K, which pipelines its
+  // Items beyond the clusters' reach, in at most two waves: one CTA per whole
+  // item has no item boundary inside a CTA's range and no merge, but every
+  // wave pays a cold start.  Taken when that makespan is no longer than
+  // stream-K's share plus one start, its end merge and two boundaries.  With
+  // more waves the starts add up and persistent stream-K, which pipelines its
   // loads across item boundaries, wins (measured: 2048 items, 649 -> 705 us).
   q.whole_items = false;
-  if (q.cs == 0 && q.items > num_sms) {
+  if (q.cs == 0 && q.items * 2 > num_sms) {
     const long long waves = (q.items + num_sms - 1) / num_sms;
-    const double sk_tiles = (double)q.total_units / num_sms + 2 * kBoundaryTiles;
-    q.whole_items = waves <= 2 && (double)(waves * q.tpi) <= sk_tiles;
+    const double whole = (double)waves * (q.tpi + kStartTiles);
+    const double sk = (double)q.total_units / num_sms + kStartTiles + kMergeTiles + 2 * kBoundaryTiles;
+    q.whole_items = waves <= 2 && whole <= sk;
   }
   q.partial_bytes = align_up((size_t)q.grid * 2 * ((size_t)q.NQ * dh + 2 * q.NQ) * sizeof(float), 256);
   q.counter_bytes = align_up((size_t)q.items * sizeof(unsigned), 256);

@@ -79,9 +79,9 @@ def test_ragged_shapes(F, dtype, dh, shape):
 
 
 # (B, N, D, H, dh, nq, work split the attention must take on 148 SMs); items =
-# B * H * query chunks of up to 64 rows.  Whole-item mode takes SMs < items <=
-# 2 SMs when its two waves are no slower than stream-K; stream-K takes the rest
-# above SMs / 2.
+# B * H * query chunks of up to 64 rows.  Above SMs / 2 items, whole-item mode
+# takes one or two waves when they are no slower than stream-K's share plus its
+# merge and boundaries; stream-K takes the rest.
 SPLIT_SHAPES = [
     pytest.param(9, 1000, 128, 32, 64, 20, "whole", id="whole-288items-nq32-dh64"),
     pytest.param(9, 700, 128, 32, 128, 12, "whole", id="whole-288items-nq16-dh128"),
@@ -91,10 +91,13 @@ SPLIT_SHAPES = [
     pytest.param(12, 700, 128, 16, 128, 12, "stream", id="streamk-192items-nq16-dh128"),
     pytest.param(8, 1024, 128, 32, 128, 32, "stream", id="streamk-256items-nq32-dh128"),
     pytest.param(5, 1000, 128, 32, 128, 40, "stream", id="streamk-160items-nq48-dh128"),
-    pytest.param(3, 900, 128, 32, 128, 60, "stream", id="streamk-96items-nq64-dh128"),
-    pytest.param(3, 900, 128, 32, 64, 44, "stream", id="streamk-96items-nq48-dh64"),
+    pytest.param(3, 900, 128, 32, 128, 60, "whole", id="whole-96items-nq64-dh128"),
+    pytest.param(3, 900, 128, 32, 64, 44, "whole", id="whole-96items-nq48-dh64"),
+    pytest.param(2, 800, 128, 32, 64, 100, "whole", id="whole-128items-2chunks-dh64"),
+    pytest.param(5, 900, 128, 32, 128, 60, "stream", id="streamk-160items-nq64-dh128"),
+    pytest.param(5, 900, 128, 32, 64, 44, "stream", id="streamk-160items-nq48-dh64"),
     pytest.param(12, 600, 128, 32, 64, 30, "stream", id="streamk-384items-nq32-dh64"),
-    pytest.param(2, 800, 128, 32, 64, 100, "stream", id="streamk-128items-2chunks-dh64"),
+    pytest.param(5, 800, 128, 32, 64, 100, "stream", id="streamk-320items-2chunks-dh64"),
     pytest.param(16, 1024, 128, 32, 128, 32, "stream", id="streamk-512items-nq32-dh128"),
 ]
 _SPLIT_CODE = {"stream": 1, "whole": 2, "cluster": 3}
@@ -118,8 +121,8 @@ def test_attention_work_splits(F, B, N, D, H, dh, nq, split):
     _check_fused(F, inp, seqs_for_oracle=seqs)
 
 
-@pytest.mark.parametrize("B,N,D,H,dh,nq", [(12, 600, 128, 32, 64, 30), (3, 900, 128, 32, 128, 40),
-                                            (3, 900, 128, 32, 128, 60)])
+@pytest.mark.parametrize("B,N,D,H,dh,nq", [(12, 600, 128, 32, 64, 30), (5, 900, 128, 32, 128, 40),
+                                            (5, 900, 128, 32, 128, 60)])
 def test_stream_k_deterministic(F, B, N, D, H, dh, nq):
     """Stream-K merges a split item in CTA order by its last contributor: two
     runs give the same bits whatever order the contributors finish in."""

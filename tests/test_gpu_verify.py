@@ -68,12 +68,15 @@ _SPLIT_CODE = {"stream": 1, "whole": 2, "cluster": 3}
 # (B, N, D, H, dh, |T_v|, |S|, split the attention must take on 148 SMs):
 # R = |T_v| + 2 |S| rows per sequence, query chunks of 16, 32 or 64 rows
 VERIFY_SPLITS = [
-    pytest.param(3, 700, 128, 32, 128, 4, 6, "stream", id="streamk-96items-nq16-dh128"),
-    pytest.param(3, 700, 128, 32, 128, 6, 12, "stream", id="streamk-96items-nq32-dh128"),
-    pytest.param(3, 700, 128, 32, 128, 8, 20, "stream", id="streamk-96items-nq48-dh128"),
-    pytest.param(3, 700, 128, 32, 128, 8, 26, "stream", id="streamk-96items-nq64-dh128"),
-    pytest.param(3, 700, 128, 32, 64, 8, 20, "stream", id="streamk-96items-nq48-dh64"),
-    pytest.param(2, 700, 128, 32, 128, 20, 40, "stream", id="streamk-128items-2chunks-dh128"),
+    pytest.param(5, 700, 128, 32, 128, 4, 6, "stream", id="streamk-160items-nq16-dh128"),
+    pytest.param(5, 700, 128, 32, 128, 6, 12, "stream", id="streamk-160items-nq32-dh128"),
+    pytest.param(5, 700, 128, 32, 128, 8, 20, "stream", id="streamk-160items-nq48-dh128"),
+    pytest.param(5, 700, 128, 32, 128, 8, 26, "stream", id="streamk-160items-nq64-dh128"),
+    pytest.param(5, 700, 128, 32, 64, 8, 20, "stream", id="streamk-160items-nq48-dh64"),
+    pytest.param(5, 700, 128, 32, 128, 20, 40, "stream", id="streamk-320items-2chunks-dh128"),
+    pytest.param(3, 700, 128, 32, 128, 4, 6, "whole", id="whole-96items-nq16-dh128"),
+    pytest.param(3, 700, 128, 32, 128, 8, 26, "whole", id="whole-96items-nq64-dh128"),
+    pytest.param(2, 700, 128, 32, 128, 20, 40, "whole", id="whole-128items-2chunks-dh128"),
     pytest.param(5, 1000, 128, 32, 128, 8, 16, "stream", id="streamk-160items-nq48-dh128"),
     pytest.param(5, 1000, 128, 32, 128, 8, 26, "stream", id="streamk-160items-nq64-dh128"),
     pytest.param(9, 1000, 128, 32, 128, 8, 16, "whole", id="whole-288items-nq48-dh128"),
@@ -101,7 +104,7 @@ def test_verify_work_splits(F, B, N, D, H, dh, n_tv, n_s, split, causal):
 @pytest.mark.parametrize("causal", [False, True], ids=["mutual", "causal"])
 def test_verify_stream_k_deterministic(F, causal):
     """Two stream-K verify passes on the same inputs give the same bits."""
-    B, N, D, H, dh, n_tv, n_s = 3, 700, 128, 32, 128, 8, 20
+    B, N, D, H, dh, n_tv, n_s = 5, 700, 128, 32, 128, 8, 20
     _assert_split(F, B, N, H, dh, n_tv + 2 * n_s, n_s, "stream")
     inp = W.random_verify(B, N, D, H, dh, n_tv=n_tv, n_s=n_s, seed=67)
     a, b = W.to_device(inp), W.to_device(inp)
