@@ -16,14 +16,16 @@
 // are then rescaled), so most tiles need no rescaling; P goes to shared memory
 // as bf16 in the MN-major swizzled layout the PV MMA reads.
 //
-// Two ways to spread the units (item = (sequence, head, query chunk), 128-key
-// tile) over the SMs:
-//   cluster mode (few items): one thread-block cluster of cs <= 8 CTAs per
-//     item, each CTA an equal share of its tiles.  The CTAs leave their (O, m,
-//     l) partials in their own shared memory and, after a cluster barrier,
-//     each merges a slice of the head dimension reading the others' partials
-//     through distributed shared memory.
-//   persistent stream-K (many items): one CTA per SM; units are laid out item
+// Three ways to spread the units (item = (sequence, head, query chunk),
+// 128-key tile) over the SMs:
+//   cluster mode (at most SMs/2 items): one thread-block cluster of cs <= 8
+//     CTAs per item, each CTA an equal share of its tiles.  The CTAs leave
+//     their (O, m, l) partials in their own shared memory and, after a cluster
+//     barrier, each merges a slice of the head dimension reading the others'
+//     partials through distributed shared memory.
+//   whole items (up to two waves, when no slower by the plan's cost model):
+//     one CTA per item, no merge.
+//   persistent stream-K (the rest): one CTA per SM; units are laid out item
 //     after item and every CTA takes an equal contiguous range, so the cache
 //     stream is balanced whatever B, H, N.  An item split between CTAs leaves
 //     (O, m, l) partials in global memory; its last contributor (atomic
@@ -37,9 +39,9 @@
 //
 // The O^T accumulator is double-buffered in TMEM by segment (the tiles of one
 // item in a CTA's range), so a segment's end costs the softmax warps only the
-// reduction of l: its output or partial is written two tiles later, once its
-// last PV is long done, while the next segment's PVs accumulate in the other
-// buffer.  A partial's writers signal the finisher, which fences and takes the
+// reduction of l: its output or partial is written at the end of a later tile,
+// once its last PV is done, while the next segment's PVs accumulate in the
+// other buffer.  A partial's writers signal the finisher, which fences and takes the
 // item count off the softmax warps' path; the items this CTA completes last
 // are merged after its range.
 //
