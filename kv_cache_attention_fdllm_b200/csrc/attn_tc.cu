@@ -185,10 +185,25 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// w (16, or 8 for the last chunk of 24 columns) columns of this thread's TMEM
+// row; w is a constant once the caller's loop is unrolled
+__device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, float* v, int w) {
+  if (w >= 16)
+    tc::tmem_ld16(taddr, v);
+  else
+    tc::tmem_ld8(taddr, v);
+}
+__device__ __forceinline__ void tmem_st_chunk(uint32_t taddr, const float* v, int w) {
+  if (w >= 16)
+    tc::tmem_st16(taddr, v);
+  else
+    tc::tmem_st8(taddr, v);
+}
+
 template <int NQ>
 __device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float* v) {
 #pragma unroll
-  for (int c = 0; c < NQ; c += 16) tc::tmem_ld16(taddr + c, v + c);
+  for (int c = 0; c < NQ; c += 16) tmem_ld_chunk(taddr + c, v + c, NQ - c < 16 ? NQ - c : 16);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -216,12 +231,13 @@ struct Smem {
 };
 
 // Softmax threads: NQ/kCols groups of 4 warps; a thread owns one key (one dh
-// row) and kCols query columns (16, or 32 at NQ = 64: 256 threads whose
-// registers hold a tile's 32 scores without spilling).  One more warp, the
-// finisher, takes the item counts of the partial segments.
+// row) and kCols query columns: 16, or 24 at NQ = 48 and 32 at NQ = 64, so that
+// those run 8 softmax warps, whose registers hold a tile's scores without
+// spilling.  One more warp, the finisher, takes the item counts of the partial
+// segments.
 template <int NQ>
 struct Threads {
-  static constexpr int kCols = NQ == 64 ? 32 : 16;
+  static constexpr int kCols = NQ == 64 ? 32 : (NQ == 48 ? 24 : 16);
   static constexpr int kSmx = 128 * NQ / kCols;
   static constexpr int kFinisher = 2 + kSmx / 32;  // warp index
   static constexpr int kAll = 64 + kSmx + 32;
@@ -540,12 +556,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (t0 == 0 && tl == tpi - 1) {
 #pragma unroll
         for (int cc = 0; cc < NQH; cc += 16) {
+          const int w = NQH - cc < 16 ? NQH - cc : 16;
           float o[16];
-          tc::tmem_ld16(t_o + cc, o);
+          tmem_ld_chunk(t_o + cc, o, w);
           tc::tmem_wait_ld();
           if (kl < DH) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
+            for (int c = 0; c < w; ++c) {
               const int cq = c0 + cc + c, r = qc * NQ + cq;
               if (r < p.rows) {
                 const float lt = sls[cq];
@@ -562,14 +579,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float* part = p.partials + ((size_t)cta * 2 + slot) * part_floats;
 #pragma unroll
         for (int cc = 0; cc < NQH; cc += 16) {
+          const int w = NQH - cc < 16 ? NQH - cc : 16;
           float o[16];
-          tc::tmem_ld16(t_o + cc, o);
+          tmem_ld_chunk(t_o + cc, o, w);
           tc::tmem_wait_ld();
           if (kl < DH) {
-            // O as [dh row][NQ columns]: a thread's 16 columns are 64 contiguous bytes
+            // O as [dh row][NQ columns]: a thread's columns are contiguous
             float4* dst = reinterpret_cast<float4*>(part + (size_t)kl * NQ + c0 + cc);
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
+            for (int v = 0; v < w / 4; ++v)
               dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
           }
         }
@@ -764,11 +782,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float o[16];
 #pragma unroll
         for (int cc = 0; cc < NQH; cc += 16) {
-          tc::tmem_ld16(t_oc + lane_off + c0 + cc, o);
+          const int w = NQH - cc < 16 ? NQH - cc : 16;
+          tmem_ld_chunk(t_oc + lane_off + c0 + cc, o, w);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 16; ++c) o[c] *= alpha[c0 + cc + c];
-          tc::tmem_st16(t_oc + lane_off + c0 + cc, o);
+          for (int c = 0; c < w; ++c) o[c] *= alpha[c0 + cc + c];
+          tmem_st_chunk(t_oc + lane_off + c0 + cc, o, w);
         }
         tc::tmem_wait_st();
       }
@@ -874,13 +893,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       float* cpart = reinterpret_cast<float*>(k_ring);
 #pragma unroll
       for (int cc = 0; cc < NQH; cc += 16) {
+        const int w = NQH - cc < 16 ? NQH - cc : 16;
         float o[16];
-        tc::tmem_ld16(tmem_o + lane_off + c0 + cc, o);
+        tmem_ld_chunk(tmem_o + lane_off + c0 + cc, o, w);
         tc::tmem_wait_ld();
         if (kl < DH) {
           float4* dst = reinterpret_cast<float4*>(cpart + kl * kP + c0 + cc);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          for (int v = 0; v < w / 4; ++v)
+            dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
         }
       }
       if (st < NQ) {
@@ -1016,7 +1037,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         if (st < NQ && p.lse && qc * NQ + st < p.rows)
           p.lse[((size_t)b * p.rows + qc * NQ + st) * p.H + h] = M + log2f(Lsum);
-        constexpr int kJ = NQH == 32 ? 2 : 4;  // contributors per batch of O loads
+        constexpr int kJ = NQH >= 24 ? 2 : 4;  // contributors per batch of O loads
         float acc[NQH];
 #pragma unroll
         for (int c = 0; c < NQH; ++c) acc[c] = 0.f;
