@@ -34,7 +34,7 @@
 //   warp 0      TMA producer: Q chunk per item, K and V tiles (128 x 64 boxes)
 //   warp 1      TMEM allocation; lane 0 issues QK (ahead by one tile) and PV
 //   warps 2..   softmax over S^T, P, accumulator rescale, epilogue: NQ/kCols
-//               groups of 4 warps (8 warps at NQ = 32 and 64, 4 at NQ = 16)
+//               groups of 4 warps (8 warps at NQ = 32, 48 and 64, 4 at NQ = 16)
 //   last warp   finisher: the item counts of partial segments (stream-K)
 //
 // The O^T accumulator is double-buffered in TMEM by segment (the tiles of one
