@@ -99,6 +99,10 @@ SPLIT_SHAPES = [
     pytest.param(12, 600, 128, 32, 64, 30, "stream", id="streamk-384items-nq32-dh64"),
     pytest.param(5, 800, 128, 32, 64, 100, "stream", id="streamk-320items-2chunks-dh64"),
     pytest.param(16, 1024, 128, 32, 128, 32, "stream", id="streamk-512items-nq32-dh128"),
+    # one- and two-tile items: a CTA's range holds several short segments, each
+    # finished while later ones run (whole ones and split ones)
+    pytest.param(16, 100, 128, 32, 128, 8, "stream", id="streamk-512items-1tile"),
+    pytest.param(16, 200, 128, 32, 64, 12, "stream", id="streamk-512items-2tiles-dh64"),
 ]
 _SPLIT_CODE = {"stream": 1, "whole": 2, "cluster": 3}
 

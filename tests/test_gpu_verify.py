@@ -81,6 +81,7 @@ VERIFY_SPLITS = [
     pytest.param(5, 1000, 128, 32, 128, 8, 26, "stream", id="streamk-160items-nq64-dh128"),
     pytest.param(9, 1000, 128, 32, 128, 8, 16, "whole", id="whole-288items-nq48-dh128"),
     pytest.param(9, 1000, 128, 32, 128, 8, 26, "whole", id="whole-288items-nq64-dh128"),
+    pytest.param(16, 100, 128, 32, 128, 4, 6, "stream", id="streamk-512items-2tiles-side"),
 ]
 
 
