@@ -267,8 +267,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint64_t* k_empty = k_full + 8;
   uint64_t* v_full = k_empty + 8;
   uint64_t* v_empty = v_full + 8;
-  uint64_t* q_full = v_empty + 8;    // [2]
-  uint64_t* q_empty = q_full + 2;    // [2]
+  uint64_t* q_full = v_empty + 8;    // [2], [0] used: the one Q buffer
+  uint64_t* q_empty = q_full + 2;    // [2], [0] used
   uint64_t* s_full = q_empty + 2;    // [2]
   uint64_t* s_empty = s_full + 2;    // [2]
   uint64_t* p_full = s_empty + 2;    // [2]
